@@ -1,0 +1,488 @@
+"""Benchmark of the sign-weight linear layers on B200 (one JSON line on rank 0).
+
+Workload (default): OneBit decode GEMV -- X M x 4096 bf16 ~N(0,1) for M in
+{1, 4, 16}, W 4096 x 4096 ~N(0, 0.02) packed to 2 MiB of signs, a, b fp32 from
+SVID.  One step = one decode token through a pool of L distinct 4096 x 4096
+OneBit layers at each batch size (for M in {1,4,16}: for each layer: ob_linear),
+so every call reads its weights from HBM: the pool (L x 2.1 MB) is larger than
+three times the L2 cache.  The step is captured once as a CUDA graph and
+replayed; inputs are resident in HBM when the timed region starts.
+
+  value     HBM GB/s of the step: algorithmic bytes (packed signs + a + b + X + Y
+            per call) / device time, summed over ranks, time = max over ranks.
+  roofline  the decode kernel: algorithmic bytes per launch / average launch
+            time, against the measured HBM copy bandwidth.
+  e2e       the same metric through the C-ABI with host buffers: pinned X is
+            copied to the device and Y back inside the timed region.
+  extra     prefill (M=2048, 4096 -> 11008, tensor-core TFLOP/s) and DBF
+            (K=N=4096, r=2048, M in {1, 512}) measured in the same run.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm of this
+build) on a bounded sample of the same workload and metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ob_linear/dbf_linear TFLOP/s-equiv & weight GB/s at M=1/16/2048, % of roofline"
+N_DIM = K_DIM = 4096
+DECODE_MS = (1, 4, 16)
+LAYERS = 192          # 192 x 2.13 MB = 409 MB of weights per pass > 3 x 126 MB L2
+SEED = 1
+
+
+def decode_call_bytes(M: int, N: int = N_DIM, K: int = K_DIM) -> int:
+    """Algorithmic HBM bytes of one OneBit call: packed signs, a, b, X (bf16), Y (bf16)."""
+    return N * K // 8 + 4 * N + 4 * K + 2 * M * K + 2 * M * N
+
+
+def step_bytes(layers: int) -> int:
+    return layers * sum(decode_call_bytes(m) for m in DECODE_MS)
+
+
+def step_flops(layers: int) -> int:
+    return layers * sum(2 * m * N_DIM * K_DIM for m in DECODE_MS)
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        import torch
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, interval_ms: int = 50):
+        self.dev = device_index
+        self.interval = interval_ms
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.interval)], stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self) -> dict:
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def ncu_traffic(kernel_file: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, or None if the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    import hashlib
+    with open(path) as f:
+        table = json.load(f)
+    entry = table.get(key)
+    if not entry:
+        return None
+    with open(os.path.join(ROOT, "binary_weight_gemm_b200", "csrc", kernel_file), "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    return entry["bytes_per_launch"] if entry.get("source_sha") == digest else None
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ reference arm (the oracle on the host)
+
+def oracle_step_sample(budget_s: float, steps: int | None = None, warmup: int = 0):
+    """Time the oracle's direct form on one 4096 x 4096 layer at M = 1, 4, 16 (one layer per step)."""
+    import oracle
+    from binary_weight_gemm_b200 import synth
+    W = synth.weights(SEED, N_DIM, K_DIM)
+    # The oracle's SVID (full SVD) is the conversion step; it is timed once, outside the linear sample.
+    t0 = time.perf_counter()
+    a, b, _ = oracle.svid_rank1(W)
+    svd_s = time.perf_counter() - t0
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    S = oracle.sign_pm1(W)
+    xs = {m: synth.activations(SEED, m, K_DIM)[1] for m in DECODE_MS}
+
+    def one():
+        for m in DECODE_MS:
+            oracle.onebit_linear(xs[m], S, a, b)
+
+    for _ in range(warmup):
+        one()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        one()
+        n += 1
+        el = time.perf_counter() - t0
+        if (steps is not None and n >= steps) or (steps is None and el >= budget_s):
+            break
+    return n, el, svd_s
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    steps = max(1, args.steps)
+    n, el, svd_s = oracle_step_sample(0.0, steps=steps, warmup=args.warmup)
+    bytes_per = step_bytes(1)
+    value = bytes_per * n / el / 1e9
+    cores = cpu_cores()
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+        "steps": n, "warmup": args.warmup, "ms_per_step": 1e3 * el / n, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "onebit_decode_4096x4096_M1_4_16", "layers_per_step": 1,
+                   "M": list(DECODE_MS), "N": N_DIM, "K": K_DIM, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} steps x (M=1,4,16) on one 4096x4096 layer, direct form "
+                                   f"(W_hat materialised each call); SVID full SVD once: {svd_s:.1f} s"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+    from binary_weight_gemm_b200 import build, synth
+    build.build()
+    from binary_weight_gemm_b200 import ops
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    peaks = load_peaks()
+    L = args.layers
+
+    # Weights: one seeded 4096 x 4096 matrix, converted by the library (pack + SVID, timed once).
+    W = torch.from_numpy(synth.weights(SEED, N_DIM, K_DIM)).to(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        P0 = ops.ob_pack_signs(W, stream=stream)
+        ev1.record(stream)
+        stream.synchronize()
+        pack_ms = ev0.elapsed_time(ev1)
+        t0 = time.perf_counter()
+        a0, b0, _, svid_iters, _ = ops.ob_svid_rank1(W, stream=stream)
+        svid_ms = 1e3 * (time.perf_counter() - t0)
+    del W
+    # Pool of L distinct weight buffers (same values, different addresses) so each call misses L2.
+    pool = [(P0.clone(), a0.clone(), b0.clone()) for _ in range(L)]
+    xs = {m: torch.from_numpy(synth.activations(SEED, m, K_DIM)[0].view(np.int16)).to(dev).view(torch.bfloat16)
+          for m in DECODE_MS}
+    ys = {m: torch.empty((m, N_DIM), dtype=torch.bfloat16, device=dev) for m in DECODE_MS}
+    torch.cuda.synchronize()
+
+    def step(s, ms=DECODE_MS):
+        for m in ms:
+            for (P, a, b) in pool:
+                ops.ob_linear(xs[m], P, a, b, out=ys[m], stream=s)
+
+    # Capture one step as a CUDA graph (calls are stream-ordered; no allocation inside).
+    with torch.cuda.stream(stream):
+        step(stream)  # warm: first calls set kernel attributes
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step(stream)
+    launches_per_step = L * len(DECODE_MS)
+
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                graph.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(end)
+    ms_max = max_over_ranks(ms, world)
+    value = world * step_bytes(L) * args.steps / (ms_max * 1e-3) / 1e9
+    tflops = world * step_flops(L) * args.steps / (ms_max * 1e-3) / 1e12
+
+    # Per-M breakdown (same graph technique, one M at a time).
+    per_m = {}
+    for m in DECODE_MS:
+        with torch.cuda.stream(stream):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(stream, ms=(m,))
+            g.replay()
+            stream.synchronize()
+            reps = max(3, args.steps // 4)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+            stream.synchronize()
+        t_call = e0.elapsed_time(e1) * 1e-3 / (reps * L)
+        per_m[str(m)] = {"us_per_call": t_call * 1e6, "hbm_gbs": decode_call_bytes(m) / t_call / 1e9,
+                         "weight_gbs": (N_DIM * K_DIM // 8 + 4 * (N_DIM + K_DIM)) / t_call / 1e9,
+                         "tflops_equiv": 2 * m * N_DIM * K_DIM / t_call / 1e12,
+                         "frac_hbm": decode_call_bytes(m) / t_call / 1e9 / peaks["hbm_gbs"]}
+        del g
+
+    # Dominant kernel: the tensor-memory decode kernel, one launch per call.
+    avg_launch_s = ms * 1e-3 / (args.steps * launches_per_step)
+    avg_bytes = step_bytes(L) / launches_per_step
+    achieved = avg_bytes / avg_launch_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                "kernel": "sign_gemm_tc_decode_kernel",
+                "traffic": ncu_traffic("linear_tc_decode.cu", "decode_4096x4096")}
+
+    # End to end through the C-ABI with host buffers: pinned X in, Y out, inside the timed region.
+    hx = {m: xs[m].cpu().pin_memory() for m in DECODE_MS}
+    hy = {m: torch.empty((m, N_DIM), dtype=torch.bfloat16).pin_memory() for m in DECODE_MS}
+    e2e_layers = min(L, 48)
+
+    def e2e_step():
+        for m in DECODE_MS:
+            for (P, a, b) in pool[:e2e_layers]:
+                xs[m].copy_(hx[m], non_blocking=True)
+                ops.ob_linear(xs[m], P, a, b, out=ys[m], stream=stream)
+                hy[m].copy_(ys[m], non_blocking=True)
+
+    e2e_steps = max(2, args.steps // 10)
+    with torch.cuda.stream(stream):
+        e2e_step()
+        stream.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        stream.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * step_bytes(e2e_layers) * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    h2d = e2e_layers * sum(2 * m * K_DIM for m in DECODE_MS)
+    d2h = e2e_layers * sum(2 * m * N_DIM for m in DECODE_MS)
+
+    extra = run_extra(ops, dev, stream, peaks) if (args.extra and world == 1) else None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, el, svd_s = oracle_step_sample(args.cpu_seconds)
+        cpu = {"value": step_bytes(1) * n / el / 1e9, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"{n} steps x (M=1,4,16) on one 4096x4096 layer in {el:.1f} s, fp64 direct form "
+                         f"(W_hat materialised per call); oracle SVID (full SVD) {svd_s:.1f} s once"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "onebit_decode_4096x4096_M1_4_16", "M": list(DECODE_MS), "N": N_DIM,
+                       "K": K_DIM, "layers_per_step": L,
+                       "l2": f"inputs larger than L2: rotating pool of {L} weight sets "
+                             f"({L * decode_call_bytes(0) / 1e6:.0f} MB) per pass",
+                       "graph": "one CUDA graph per step, programmatic dependent launch between calls",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "tflops_equiv": tflops,
+            "per_m": per_m,
+            "roofline": roofline,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "layers_per_step": e2e_layers},
+            "gpu_launches": args.steps * launches_per_step,
+            "clocks": clocks.summary(),
+            "offline": {"pack_ms": pack_ms, "svid_ms": svid_ms, "svid_iters": svid_iters,
+                        "pack_gbs": (N_DIM * K_DIM * 4 + N_DIM * K_DIM // 8) / (pack_ms * 1e-3) / 1e9},
+            "cpu_baseline": cpu,
+            "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    del graph
+
+
+def _time_calls(fn, stream, reps):
+    import torch
+    with torch.cuda.stream(stream):
+        fn(0)
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(reps):
+            fn(i)
+        e1.record(stream)
+        stream.synchronize()
+    return e0.elapsed_time(e1) * 1e-3 / reps
+
+
+def run_extra(ops, dev, stream, peaks):
+    """Prefill and DBF workloads, measured briefly in the same run (rotating buffers > L2)."""
+    import torch
+    from binary_weight_gemm_b200 import synth
+    out = {}
+    # Prefill: X 2048 x 4096, W 11008 x 4096 (5.6 MB packed), Y 2048 x 11008.
+    M, K, N = 2048, 4096, 11008
+    W = torch.from_numpy(synth.weights(2, N, K)).to(dev)
+    P = ops.ob_pack_signs(W, stream=stream)
+    a, b, _, _, _ = ops.ob_svid_rank1(W, stream=stream)
+    del W
+    sets = [(torch.from_numpy(synth.activations(2 + i, M, K)[0].view(np.int16)).to(dev).view(torch.bfloat16),
+             P.clone(), torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for i in range(3)]
+    t = _time_calls(lambda i: ops.ob_linear(sets[i % 3][0], sets[i % 3][1], a, b, out=sets[i % 3][2],
+                                            stream=stream), stream, 30)
+    fl = 2 * M * N * K
+    out["prefill_2048x4096x11008"] = {"us_per_call": t * 1e6, "tflops": fl / t / 1e12,
+                                      "frac_bf16_burst": fl / t / 1e12 / peaks["bf16_tflops"],
+                                      "frac_bf16_sustained": fl / t / 1e12 / (peaks["bf16_tflops_sustained"] or 1),
+                                      "kernel": "sign_gemm_tc_kernel"}
+    del sets
+    # DBF: K = N = 4096, r = 2048.
+    f = synth.dbf_factors(3, 4096, 2048, 4096)
+    SB = ops.ob_pack_signs(torch.from_numpy(f["S_B"].astype(np.float32)).to(dev), stream=stream)
+    SA = ops.ob_pack_signs(torch.from_numpy(f["S_A"].astype(np.float32)).to(dev), stream=stream)
+    vec = {k: torch.from_numpy(f[k]).to(dev) for k in ("a", "m", "b")}
+    for M in (1, 512):
+        nset = 64 if M == 1 else 8
+        pool = [(SB.clone(), SA.clone()) for _ in range(nset)]
+        X = torch.from_numpy(synth.activations(3, M, 4096)[0].view(np.int16)).to(dev).view(torch.bfloat16)
+        Y = torch.empty((M, 4096), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(ops.dbf_workspace_size(M, 2048), dtype=torch.uint8, device=dev)
+        t = _time_calls(lambda i: ops.dbf_linear(X, pool[i % nset][0], vec["m"], pool[i % nset][1], vec["a"],
+                                                 vec["b"], out=Y, workspace=ws, stream=stream), stream,
+                        max(50, 4 * nset))
+        fl = 2 * M * 2048 * (4096 + 4096)
+        byts = 2048 * 4096 // 8 * 2 + 4 * (4096 * 2 + 2048) + 2 * M * 4096 * 2
+        out[f"dbf_M{M}"] = {"us_per_call": t * 1e6, "tflops_equiv": fl / t / 1e12, "hbm_gbs": byts / t / 1e9,
+                            "frac_hbm": byts / t / 1e9 / peaks["hbm_gbs"],
+                            "frac_bf16_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--no-extra", dest="extra", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

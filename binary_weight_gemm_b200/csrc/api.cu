@@ -1,0 +1,253 @@
+// api.cu -- the C ABI of libobgemm (declarations and contracts in include/obgemm.h).
+//
+// Host-side argument checks, kernel dispatch and the per-device error word.
+// Checks run before any CUDA call, so a rejected call launches nothing.
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "ob_device.cuh"
+#include "ob_internal.h"
+
+// Device error word: bits OB_DEVERR_* set by kernels, read and cleared by ob_last_device_error.
+__device__ unsigned g_ob_error_word;
+
+namespace ob {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  unsigned* err = nullptr;
+  int num_sms = 0;
+  int major = 0;
+  bool ready = false;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+// Error word address, SM count and architecture of the current device (cached per device).
+ob_status current_device(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return OB_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ob_error_word) != cudaSuccess) return OB_ERR_CUDA;
+    int sms = 0, major = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return OB_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return OB_ERR_CUDA;
+    d.err = static_cast<unsigned*>(p);
+    d.num_sms = sms;
+    d.major = major;
+    d.ready = true;
+  }
+  *out = d;
+  return OB_OK;
+}
+
+bool env_flag(const char* name, bool dflt) {
+  const char* s = std::getenv(name);
+  if (!s || !*s) return dflt;
+  return !(s[0] == '0' || s[0] == 'n' || s[0] == 'N' || s[0] == 'f' || s[0] == 'F');
+}
+
+int decode_max_m() {
+  const char* s = std::getenv("OB_DECODE_MAX_M");
+  int v = s ? std::atoi(s) : kDecodeMaxM;
+  return v < 0 ? 0 : v;
+}
+
+ob_status make_ctx(void* stream, LaunchCtx* c) {
+  DeviceInfo d;
+  ob_status st = current_device(&d);
+  if (st != OB_OK) return st;
+  if (d.major != 10) return OB_ERR_UNSUPPORTED;  // sm_100 family only
+  c->stream = static_cast<cudaStream_t>(stream);
+  c->err = d.err;
+  c->num_sms = d.num_sms;
+  c->pdl = env_flag("OB_PDL", true);
+  return OB_OK;
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+ob_status zero_output(void* Y, int64_t M, int64_t N, int y_dtype, cudaStream_t s) {
+  const size_t bytes = (size_t)M * (size_t)N * (y_dtype == OB_OUT_F32 ? 4 : 2);
+  return cudaMemsetAsync(Y, 0, bytes, s) == cudaSuccess ? OB_OK : OB_ERR_CUDA;
+}
+
+ob_status status_of(cudaError_t e) {
+  if (e == cudaSuccess) return OB_OK;
+  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return OB_ERR_UNSUPPORTED;
+  return OB_ERR_CUDA;
+}
+
+ob_status run_sign_gemm(const SignGemmArgs& g, int path, const LaunchCtx& c) {
+  if (path == OB_PATH_AUTO) path = (g.M <= decode_max_m()) ? OB_PATH_TC_DECODE : OB_PATH_TC;
+  cudaError_t e;
+  switch (path) {
+    case OB_PATH_SIMT: e = launch_sign_gemm_simt(g, c); break;
+    case OB_PATH_TC_DECODE: e = launch_sign_gemm_tc_decode(g, c); break;
+    case OB_PATH_TC: e = launch_sign_gemm_tc(g, c); break;
+    default: return OB_ERR_UNSUPPORTED;
+  }
+  return status_of(e);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+}  // namespace ob
+
+using namespace ob;
+
+extern "C" {
+
+const char* ob_status_string(int status) {
+  switch (status) {
+    case OB_OK: return "OB_OK";
+    case OB_ERR_NULL: return "OB_ERR_NULL: a required pointer is NULL";
+    case OB_ERR_SHAPE: return "OB_ERR_SHAPE: negative size, or K / r not a multiple of 32";
+    case OB_ERR_ALIGN: return "OB_ERR_ALIGN: a pointer is not 16-byte aligned";
+    case OB_ERR_NAN: return "OB_ERR_NAN: NaN in an input that must be finite";
+    case OB_ERR_NOT_CONVERGED: return "OB_ERR_NOT_CONVERGED: SVID reached max_iters";
+    case OB_ERR_WORKSPACE: return "OB_ERR_WORKSPACE: workspace missing or too small";
+    case OB_ERR_CUDA: return "OB_ERR_CUDA: CUDA runtime error";
+    case OB_ERR_DEVICE_TIMEOUT: return "OB_ERR_DEVICE_TIMEOUT: a bounded wait in a kernel ran out";
+    case OB_ERR_UNSUPPORTED: return "OB_ERR_UNSUPPORTED: unsupported device, size or option";
+    case OB_ERR_DEVICE_BOUNDS: return "OB_ERR_DEVICE_BOUNDS: a kernel refused an out-of-bounds access";
+    default: return "unknown ob_status";
+  }
+}
+
+int ob_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+ob_status ob_last_device_error(void* stream) {
+  DeviceInfo d;
+  ob_status st = current_device(&d);
+  if (st != OB_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return OB_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, d.err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return OB_ERR_CUDA;
+  if (word != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(d.err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return OB_ERR_CUDA;
+  }
+  if (word & OB_DEVERR_TIMEOUT) return OB_ERR_DEVICE_TIMEOUT;
+  if (word & OB_DEVERR_BOUNDS) return OB_ERR_DEVICE_BOUNDS;
+  if (word & OB_DEVERR_NAN) return OB_ERR_NAN;
+  return OB_OK;
+}
+
+ob_status ob_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* W_packed, void* stream) {
+  if (N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
+  if (N == 0 || K == 0) return OB_OK;
+  if (!W || !W_packed) return OB_ERR_NULL;
+  if (misaligned(W) || misaligned(W_packed)) return OB_ERR_ALIGN;
+  LaunchCtx c;
+  ob_status st = make_ctx(stream, &c);
+  if (st != OB_OK) return st;
+  return status_of(launch_pack_signs(W, N, K, W_packed, c));
+}
+
+size_t ob_svid_workspace_size(int64_t N, int64_t K) {
+  if (N < 0 || K < 0) return 0;
+  return svid_workspace_bytes(N, K);
+}
+
+ob_status ob_svid_rank1(const float* W, int64_t N, int64_t K, float* a, float* b, float* sigma1, int max_iters,
+                        float tol, int* iters_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (iters_out) *iters_out = 0;
+  if (N < 0 || K < 0 || K % 4 != 0) return OB_ERR_SHAPE;
+  if (N == 0 || K == 0) return OB_OK;
+  if (!W || !a || !b) return OB_ERR_NULL;
+  if (misaligned(W) || misaligned(a) || misaligned(b)) return OB_ERR_ALIGN;
+  if (!workspace || ws_bytes < svid_workspace_bytes(N, K)) return OB_ERR_WORKSPACE;
+  if (misaligned(workspace)) return OB_ERR_ALIGN;
+  if (max_iters <= 0) max_iters = 200;
+  if (!(tol > 0.f)) tol = 1e-6f;
+  LaunchCtx c;
+  ob_status st = make_ctx(stream, &c);
+  if (st != OB_OK) return st;
+  return run_svid(W, N, K, a, b, sigma1, max_iters, tol, iters_out, workspace, c);
+}
+
+ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,
+                       const float* b, void* Y, int y_dtype, int path, void* stream) {
+  if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
+  if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
+  if (path < OB_PATH_AUTO || path > OB_PATH_TC) return OB_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return OB_OK;
+  if (!Y || !a) return OB_ERR_NULL;
+  if (K > 0 && (!X || !W_packed || !b)) return OB_ERR_NULL;
+  if (misaligned(Y) || misaligned(a) || (K > 0 && (misaligned(X) || misaligned(W_packed) || misaligned(b))))
+    return OB_ERR_ALIGN;
+  LaunchCtx c;
+  ob_status st = make_ctx(stream, &c);
+  if (st != OB_OK) return st;
+  if (K == 0) return zero_output(Y, M, N, y_dtype, c.stream);
+  SignGemmArgs g{static_cast<const uint16_t*>(X), M, K, W_packed, N, b, a, Y, N, y_dtype};
+  return run_sign_gemm(g, path, c);
+}
+
+ob_status ob_linear(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,
+                    const float* b, void* Y, int y_dtype, void* stream) {
+  return ob_linear_ex(X, M, K, W_packed, N, a, b, Y, y_dtype, OB_PATH_AUTO, stream);
+}
+
+size_t dbf_workspace_size(int64_t M, int64_t r) {
+  if (M < 0 || r < 0) return 0;
+  return align256((size_t)M * (size_t)r * 2);
+}
+
+ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_packed, int64_t r, const float* m,
+                        const uint32_t* SA_packed, int64_t N, const float* a, const float* b, void* Y, int y_dtype,
+                        void* workspace, size_t ws_bytes, int path, void* stream) {
+  if (M < 0 || N < 0 || K < 0 || r < 0 || K % 32 != 0 || r % 32 != 0) return OB_ERR_SHAPE;
+  if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
+  if (path < OB_PATH_AUTO || path > OB_PATH_TC) return OB_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return OB_OK;
+  if (!Y || !a) return OB_ERR_NULL;
+  const bool empty_sum = (K == 0 || r == 0);
+  if (!empty_sum && (!X || !SB_packed || !m || !SA_packed || !b)) return OB_ERR_NULL;
+  if (misaligned(Y) || misaligned(a)) return OB_ERR_ALIGN;
+  if (!empty_sum && (misaligned(X) || misaligned(SB_packed) || misaligned(m) || misaligned(SA_packed) ||
+                     misaligned(b)))
+    return OB_ERR_ALIGN;
+  if (!empty_sum) {
+    if (!workspace || ws_bytes < dbf_workspace_size(M, r)) return OB_ERR_WORKSPACE;
+    if (misaligned(workspace)) return OB_ERR_ALIGN;
+  }
+  LaunchCtx c;
+  ob_status st = make_ctx(stream, &c);
+  if (st != OB_OK) return st;
+  if (empty_sum) return zero_output(Y, M, N, y_dtype, c.stream);
+  // T = ((X ⊙ b^T) S_B^T) ⊙ m^T, rounded once to bf16, then Y = (T S_A^T) ⊙ a^T.
+  uint16_t* T = static_cast<uint16_t*>(workspace);
+  SignGemmArgs g1{static_cast<const uint16_t*>(X), M, K, SB_packed, r, b, m, T, r, OB_OUT_BF16};
+  st = run_sign_gemm(g1, path, c);
+  if (st != OB_OK) return st;
+  SignGemmArgs g2{T, M, r, SA_packed, N, nullptr, a, Y, N, y_dtype};
+  return run_sign_gemm(g2, path, c);
+}
+
+ob_status dbf_linear(const void* X, int64_t M, int64_t K, const uint32_t* SB_packed, int64_t r, const float* m,
+                     const uint32_t* SA_packed, int64_t N, const float* a, const float* b, void* Y, int y_dtype,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  return dbf_linear_ex(X, M, K, SB_packed, r, m, SA_packed, N, a, b, Y, y_dtype, workspace, ws_bytes,
+                       OB_PATH_AUTO, stream);
+}
+
+ob_status ob_selftest_timeout(uint64_t limit_ns, void* stream) {
+  LaunchCtx c;
+  ob_status st = make_ctx(stream, &c);
+  if (st != OB_OK) return st;
+  if (launch_timeout_selftest(limit_ns, c) != cudaSuccess) return OB_ERR_CUDA;
+  return ob_last_device_error(stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,311 @@
+// linear_tc.cu -- large-M sign product on the fifth-generation tensor core.
+//
+//   Y[m, n] = oscale[n] * sum_k x[m, k] * (iscale[k] * s[n, k])
+//
+// "1bit量化" (blog.zerodtree.com), "proposition 1": [(X ⊙ b^T) W_sign^T] ⊙ a^T,
+// computed here with b folded into the sign operand (X ⊙ b^T) S^T = X (S ⊙ 1 b^T)^T;
+// "Addition is almost all you need ..." (gist.science), "Methodologie": each of
+// DBF's two sign products is one call.
+//
+// Persistent, warp-specialised kernel, one CTA per SM, output tile 128 weight
+// rows x 256 tokens:
+//  * warp 8 (one lane): TMA loads of the activation tile (256 tokens x 64 k,
+//    bf16, 128-byte swizzle) into a 4-deep shared-memory ring.  This is the MMA's
+//    B operand; the activations are never touched by a thread.
+//  * warps 0-3: one thread per weight row expands two packed words (64 k) into
+//    32 TMEM columns of bf16 pairs (+/-bf16(b_k), +/-bf16(b_k+1)) with
+//    tcgen05.st.  This is the MMA's A operand in tensor memory, so the expanded
+//    signs cost no shared-memory bandwidth.
+//  * warp 9 (one lane): tcgen05.mma kind::f16, M=128, N=256, K=16, fp32
+//    accumulators in TMEM (256 columns); tcgen05.commit releases ring slots.
+//  * warps 4-7: epilogue, tcgen05.ld of the accumulator, * oscale, bf16/fp32
+//    stores (each warp store covers 32 consecutive outputs of one token row).
+// Every mbarrier wait is bounded (see ob_device.cuh).
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+
+#include "ob_device.cuh"
+#include "ob_internal.h"
+
+namespace ob {
+namespace {
+
+constexpr int kRows = 128;     // MMA M (weight rows)
+constexpr int kTok = 256;      // MMA N (tokens)
+constexpr int kBK = 64;        // k per stage
+constexpr int kStages = 4;
+constexpr int kThreads = 320;  // 10 warps
+constexpr uint32_t kXStageBytes = kTok * kBK * 2;  // 32 KB
+constexpr int kTmemCols = 512;                     // D [0,256), A slots 256 + 32*s
+constexpr uint32_t kIdesc = idesc_bf16_f32(kRows, kTok);
+constexpr int64_t kMaxK = 24576;                   // iscale pairs staged in shared memory
+
+struct __align__(128) TcShared {  // 128-byte size keeps the bf16x2 table after it 16-byte aligned
+  uint64_t xfull[kStages];
+  uint64_t afull[kStages];
+  uint64_t empty[kStages];
+  uint64_t dfull;
+  uint64_t dempty;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, unsigned* err, volatile int* abort_flag,
+                                          int lane) {
+  int okw = 1;
+  if (lane == 0) okw = mbar_wait(bar, parity, err, abort_flag) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, okw, 0) != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                                                                    SignGemmArgs g, unsigned* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  TcShared* sh = reinterpret_cast<TcShared*>(xs + (size_t)kStages * kXStageBytes);
+  uint32_t* bpair = reinterpret_cast<uint32_t*>(sh + 1);  // [K/2] bf16x2 (iscale[2i], iscale[2i+1])
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t K = g.K, Wd = K / 32;
+  const int nkb = (int)((K + kBK - 1) / kBK);
+  const int64_t m_blocks = (g.M + kTok - 1) / kTok;
+  const int64_t n_blocks = (g.R + kRows - 1) / kRows;
+  const int64_t tiles = m_blocks * n_blocks;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh->xfull[s], 1);
+      mbar_init(&sh->afull[s], 4);
+      mbar_init(&sh->empty[s], 1);
+    }
+    mbar_init(&sh->dfull, 1);
+    mbar_init(&sh->dempty, 4);
+    sh->abort_flag = 0;
+    fence_mbar_init();
+  }
+  // Input-scale pairs as bf16x2 (round to nearest even); ones without a scale.
+  for (int64_t i = tid; i < (K + 1) / 2; i += kThreads) {
+    const float lo = g.iscale ? __ldg(g.iscale + 2 * i) : 1.f;
+    const float hi = g.iscale ? __ldg(g.iscale + 2 * i + 1) : 1.f;
+    bpair[i] = pack_bf16x2(lo, hi);
+  }
+  if (warp == 9) {
+    tmem_alloc(&sh->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  volatile int* abort_flag = &sh->abort_flag;
+  pdl_launch_dependents();
+
+  if (warp < 4) {
+    // ------------------------------------------------ A producer: signs (x) input scale -> TMEM
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    int64_t gstage = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      const int64_t n = (tile % n_blocks) * kRows + tid;
+      const bool row_ok = n < g.R;
+      const uint32_t* srow = g.S + (row_ok ? n : 0) * Wd;
+      uint32_t nw0 = row_ok ? __ldg(srow) : 0u;
+      uint32_t nw1 = (row_ok && Wd > 1) ? __ldg(srow + 1) : 0u;
+      for (int kb = 0; kb < nkb; ++kb, ++gstage) {
+        const uint32_t w0 = nw0, w1 = nw1;
+        const int64_t wn = 2 * (int64_t)(kb + 1);  // prefetch the next stage's words
+        nw0 = (row_ok && wn < Wd) ? __ldg(srow + wn) : 0u;
+        nw1 = (row_ok && wn + 1 < Wd) ? __ldg(srow + wn + 1) : 0u;
+        const int s = (int)(gstage % kStages);
+        if (gstage >= kStages) {
+          ok = wait_warp(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag, lane);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        const uint4* bp = reinterpret_cast<const uint4*>(bpair + (int64_t)kb * (kBK / 2));
+        const bool full_stage = (int64_t)(kb + 1) * kBK <= K;
+        uint32_t v[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint4 b4 = make_uint4(0, 0, 0, 0);
+          if (full_stage || q < 4) b4 = bp[q];  // a trailing half stage reads 32 k only
+          const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = q * 4 + e;          // column: k = 2c, 2c+1 within the stage
+            const uint32_t w = c < 16 ? w0 : w1;
+            const int i = (2 * c) & 31;       // bit of k = 2c
+            const uint32_t lo = i <= 15 ? (w << (15 - i)) : (w >> (i - 15));
+            const uint32_t hi = w << (30 - i);
+            v[c] = bb[e] ^ (lo & 0x8000u) ^ (hi & 0x80000000u);
+          }
+        }
+        tmem_st_x32(lane_base + 256u + 32u * s, v);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->afull[s]);
+      }
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------ epilogue
+    const int q = warp - 4;  // TMEM lane quadrant
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    pdl_wait();
+    int64_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+      if (!wait_warp(&sh->dfull, (uint32_t)it & 1u, err, abort_flag, lane)) break;
+      tc_fence_after();
+      const int64_t m0 = (tile / n_blocks) * kTok;
+      const int64_t n = (tile % n_blocks) * kRows + q * 32 + lane;
+      const bool row_ok = n < g.R;
+      const float sc = row_ok ? __ldg(g.oscale + n) : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < kTok / 32; ++c) {
+        uint32_t d[32];
+        tmem_ld_x32(lane_base + 32u * c, d);
+        tmem_wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int64_t m = m0 + 32 * c + i;
+            if (m < g.M) {
+              const float y = __uint_as_float(d[i]) * sc;
+              const int64_t off = m * g.ldy + n;
+              if (g.y_dtype == OB_OUT_F32)
+                static_cast<float*>(g.Y)[off] = y;
+              else
+                static_cast<__nv_bfloat16*>(g.Y)[off] = __float2bfloat16_rn(y);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->dempty);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap_x);
+      pdl_wait();
+      int64_t gstage = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        const int32_t m0 = (int32_t)((tile / n_blocks) * kTok);
+        for (int kb = 0; kb < nkb; ++kb, ++gstage) {
+          const int s = (int)(gstage % kStages);
+          if (gstage >= kStages) {
+            ok = mbar_wait(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag);
+            if (!ok) break;
+          }
+          mbar_arrive_expect_tx(&sh->xfull[s], kXStageBytes);
+          tma_load_2d(xs + (size_t)s * kXStageBytes, &tmap_x, &sh->xfull[s], kb * kBK, m0);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int64_t gstage = 0, it = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++it) {
+        if (it > 0) {
+          ok = mbar_wait(&sh->dempty, (uint32_t)(it - 1) & 1u, err, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        for (int kb = 0; kb < nkb; ++kb, ++gstage) {
+          const int s = (int)(gstage % kStages);
+          const uint32_t par = (uint32_t)(gstage / kStages) & 1u;
+          ok = mbar_wait(&sh->xfull[s], par, err, abort_flag) && mbar_wait(&sh->afull[s], par, err, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t xa = smem_u32(xs) + (uint32_t)s * kXStageBytes;
+          const int ksub = ((int64_t)(kb + 1) * kBK <= K) ? 4 : 2;
+          for (int q = 0; q < ksub; ++q)
+            mma_bf16_ts(tmem, tmem + 256u + 32u * s + 8u * q, sdesc_kmajor_sw128(xa + 32u * q), kIdesc,
+                        (kb > 0 || q > 0) ? 1u : 0u);
+          mma_commit(&sh->empty[s]);
+        }
+        mma_commit(&sh->dfull);
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host: tensor map
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
+  if (g.M == 0 || g.R == 0 || g.K == 0) return cudaSuccess;
+  if (g.K > kMaxK) return cudaErrorInvalidValue;
+  EncodeTiledFn encode = get_encode_fn();
+  if (!encode) return cudaErrorNotSupported;
+
+  CUtensorMap tmap;
+  std::memset(&tmap, 0, sizeof(tmap));
+  const cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.M};
+  const cuuint64_t strides[1] = {(cuuint64_t)g.K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kTok};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(g.X), dims, strides, box,
+                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+  const int64_t tiles = ((g.M + kTok - 1) / kTok) * ((g.R + kRows - 1) / kRows);
+  const int grid = (int)std::min<int64_t>(tiles, c.num_sms);
+  const size_t smem = 1024 + (size_t)kStages * kXStageBytes + sizeof(TcShared) + sizeof(uint32_t) * ((g.K + 1) / 2);
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  int na = 0;
+  if (c.pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    na = 1;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaFuncSetAttribute(sign_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  e = cudaLaunchKernelEx(&cfg, sign_gemm_tc_kernel, tmap, g, c.err);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace ob

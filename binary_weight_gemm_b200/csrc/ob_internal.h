@@ -1,0 +1,50 @@
+// ob_internal.h -- host-side launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "obgemm.h"
+
+namespace ob {
+
+struct LaunchCtx {
+  cudaStream_t stream;
+  unsigned* err;   // device error word of the current device
+  int num_sms;     // multiprocessors of the current device
+  bool pdl;        // launch with programmatic stream serialization
+};
+
+// One sign-product layer  Y[m, n] = oscale[n] * sum_k (x[m, k] * iscale[k]) * s[n, k],
+// with s the packed sign matrix (R x K, R = output features).  X is bf16 M x K
+// (row stride K); iscale may be null (no input scale).  Y is M x R with row
+// stride ldy, bf16 or fp32.
+struct SignGemmArgs {
+  const uint16_t* X;
+  int64_t M, K;
+  const uint32_t* S;
+  int64_t R;
+  const float* iscale;  // [K] or null
+  const float* oscale;  // [R]
+  void* Y;
+  int64_t ldy;
+  int y_dtype;          // ob_out_dtype
+};
+
+cudaError_t launch_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* out, const LaunchCtx& c);
+
+cudaError_t launch_sign_gemm_simt(const SignGemmArgs& g, const LaunchCtx& c);
+cudaError_t launch_sign_gemm_tc_decode(const SignGemmArgs& g, const LaunchCtx& c);
+cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c);
+
+// SVID power iteration pieces (see svid.cu).
+size_t svid_workspace_bytes(int64_t N, int64_t K);
+ob_status run_svid(const float* W, int64_t N, int64_t K, float* a, float* b, float* sigma1, int max_iters,
+                   float tol, int* iters_out, void* ws, const LaunchCtx& c);
+
+cudaError_t launch_timeout_selftest(uint64_t limit_ns, const LaunchCtx& c);
+
+// Largest M handled by one pass of the tensor-memory decode kernel.
+constexpr int kDecodeMaxM = 16;
+
+}  // namespace ob

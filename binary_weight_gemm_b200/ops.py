@@ -1,0 +1,148 @@
+"""Python binding of libobgemm: the C-ABI calls, by the same names, on torch CUDA tensors.
+
+Argument marshalling only.  Every step of the computation runs in the library's
+CUDA kernels; torch supplies device memory and the current stream.  There is no
+CPU fallback: without the built library the calls raise.
+
+Layouts (see include/obgemm.h): X bf16 [M, K]; packed signs int32 [R, C/32]
+(uint32 bit patterns, bit i of word w <-> column 32w+i, set bit = -1); scale
+vectors fp32; Y bf16 or fp32 [M, N].
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC,  # noqa: F401
+                   OB_PATH_TC_DECODE, ObError)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple | None = None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _out_code(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
+        return OB_OUT_BF16
+    if dtype == torch.float32:
+        return OB_OUT_F32
+    raise TypeError("output dtype must be torch.bfloat16 or torch.float32")
+
+
+def ob_pack_signs(W: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Packed W_sign (int32 [N, K/32]) of fp32 W [N, K]; K % 32 == 0."""
+    N, K = W.shape
+    _need(W, "W", torch.float32)
+    if out is None:
+        out = torch.empty((N, K // 32), dtype=torch.int32, device=W.device)
+    _need(out, "out", torch.int32, (N, K // 32))
+    _lib.check("ob_pack_signs", _lib.lib().ob_pack_signs(_ptr(W), N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def ob_last_device_error(stream=None) -> int:
+    """Synchronise, then read and clear the device error word (returns an ob_status code)."""
+    return int(_lib.lib().ob_last_device_error(_stream(stream)))
+
+
+def ob_svid_workspace_size(N: int, K: int) -> int:
+    return int(_lib.lib().ob_svid_workspace_size(N, K))
+
+
+def ob_svid_rank1(W: torch.Tensor, max_iters: int = 0, tol: float = 0.0, workspace: torch.Tensor | None = None,
+                  stream=None, check: bool = True):
+    """Rank-1 SVID of |W|: returns (a [N], b [K], sigma1 [1], iterations, status)."""
+    N, K = W.shape
+    _need(W, "W", torch.float32)
+    a = torch.empty(N, dtype=torch.float32, device=W.device)
+    b = torch.empty(K, dtype=torch.float32, device=W.device)
+    sigma = torch.empty(1, dtype=torch.float32, device=W.device)
+    ws_bytes = ob_svid_workspace_size(N, K)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=W.device)
+    iters = ctypes.c_int(0)
+    st = int(_lib.lib().ob_svid_rank1(_ptr(W), N, K, _ptr(a), _ptr(b), _ptr(sigma), int(max_iters),
+                                      float(tol), ctypes.byref(iters), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)))
+    if check:
+        _lib.check("ob_svid_rank1", st)
+    return a, b, sigma, iters.value, st
+
+
+def ob_linear(X: torch.Tensor, W_packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor,
+              out_dtype: torch.dtype = torch.bfloat16, path: int = OB_PATH_AUTO, out: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """OneBit layer Y = [(X ⊙ b^T) W_sign^T] ⊙ a^T; X bf16 [M, K], W_packed int32 [N, K/32]."""
+    M, K = X.shape
+    N = W_packed.shape[0]
+    _need(X, "X", torch.bfloat16)
+    _need(W_packed, "W_packed", torch.int32, (N, K // 32))
+    _need(a, "a", torch.float32, (N,))
+    _need(b, "b", torch.float32, (K,))
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    _need(out, "out", out_dtype, (M, N))
+    st = _lib.lib().ob_linear_ex(_ptr(X), M, K, _ptr(W_packed), N, _ptr(a), _ptr(b), _ptr(out),
+                                 _out_code(out_dtype), int(path), _stream(stream))
+    _lib.check("ob_linear", st)
+    return out
+
+
+def dbf_workspace_size(M: int, r: int) -> int:
+    return int(_lib.lib().dbf_workspace_size(M, r))
+
+
+def dbf_linear(X: torch.Tensor, SB_packed: torch.Tensor, m: torch.Tensor, SA_packed: torch.Tensor,
+               a: torch.Tensor, b: torch.Tensor, out_dtype: torch.dtype = torch.bfloat16,
+               path: int = OB_PATH_AUTO, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """DBF layer Y = ((((X ⊙ b^T) S_B^T) ⊙ m^T) S_A^T) ⊙ a^T.
+
+    X bf16 [M, K]; SB_packed int32 [r, K/32]; m fp32 [r]; SA_packed int32 [N, r/32].
+    """
+    M, K = X.shape
+    r = SB_packed.shape[0]
+    N = SA_packed.shape[0]
+    _need(X, "X", torch.bfloat16)
+    _need(SB_packed, "SB_packed", torch.int32, (r, K // 32))
+    _need(SA_packed, "SA_packed", torch.int32, (N, r // 32))
+    _need(m, "m", torch.float32, (r,))
+    _need(a, "a", torch.float32, (N,))
+    _need(b, "b", torch.float32, (K,))
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    _need(out, "out", out_dtype, (M, N))
+    ws_bytes = dbf_workspace_size(M, r)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=X.device)
+    st = _lib.lib().dbf_linear_ex(_ptr(X), M, K, _ptr(SB_packed), r, _ptr(m), _ptr(SA_packed), N, _ptr(a),
+                                  _ptr(b), _ptr(out), _out_code(out_dtype), _ptr(workspace), workspace.numel(),
+                                  int(path), _stream(stream))
+    _lib.check("dbf_linear", st)
+    return out
+
+
+def ob_selftest_timeout(limit_ns: int = 2_000_000, stream=None) -> int:
+    """Run the bounded-wait self-test; returns the ob_status it reports (8 = timeout recorded)."""
+    return int(_lib.lib().ob_selftest_timeout(int(limit_ns), _stream(stream)))

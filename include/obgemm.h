@@ -1,0 +1,208 @@
+/*
+ * obgemm.h -- C ABI of libobgemm.so: sign-only-weight linear layers on B200 (sm_100a).
+ *
+ * Two layer forms share one packed sign format:
+ *
+ *   OneBit  Y = [(X ⊙ b^T) · W_sign^T] ⊙ a^T
+ *           "1bit量化" (blog.zerodtree.com), notes on "OneBit: Towards Extremely
+ *           Low-bit Large Language Models": section "rank-1 approximation"
+ *           (W = W_sign ⊙ |W|, |W| ≈ a b^T) and "proposition 1".  The page
+ *           assigns b^T to the layer's input scale g and a^T to its output
+ *           scale h.
+ *
+ *   DBF     Y = ((((X ⊙ b^T) · S_B^T) ⊙ m^T) · S_A^T) ⊙ a^T
+ *           "Addition is almost all you need: Compressing large language models
+ *           with double binary factorization" (gist.science), section
+ *           "Methodologie: Double Binary Factorization (DBF)", the factorised
+ *           weight W ≈ (a ⊙ A ⊙ m^T)(B ⊙ b^T) and its inference chain.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Matrices are dense and row-major.  W is N x K (out x in), X is M x K,
+ *    Y is M x N.  Index names follow the pages: a has length N (output scale),
+ *    b has length K (input scale); for DBF, S_A is N x r, S_B is r x K, m has
+ *    length r.
+ *  - Packed sign format: row n of an R x C sign matrix is C/32 uint32 words;
+ *    bit i of word w holds column 32*w + i (least significant bit first), and
+ *    a set bit means -1, a clear bit +1.  Sign(w) = -1 exactly when w < 0, so
+ *    +0.0 and -0.0 pack as +1 (the pages leave Sign(0) open).  C must be a
+ *    multiple of 32.
+ *  - X is bf16 (IEEE bfloat16 bit patterns, passed as const void*), scale
+ *    vectors are fp32, Y is bf16 (round to nearest even) or fp32 by `y_dtype`.
+ *  - Pointers are DEVICE pointers unless a parameter says "host".  The caller
+ *    owns every buffer; the library allocates no device memory.  It holds
+ *    one 4-byte device error word per device (module-scope) and nothing else.
+ *    Every device pointer must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous and stream-ordered unless noted.
+ *  - Errors: argument checks run on the host before any launch and return a
+ *    status without launching.  Launch failures return OB_ERR_CUDA.  Faults
+ *    found on the device (a bounded wait that ran out, NaN in an input that
+ *    must be finite) set the device error word, which ob_last_device_error()
+ *    reads.  No call aborts or throws across the ABI.
+ *  - Empty problems (M == 0 or N == 0) return OB_OK and touch nothing; K == 0
+ *    (or r == 0 for DBF) writes Y = 0.
+ */
+#ifndef OBGEMM_H_
+#define OBGEMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define OB_API __attribute__((visibility("default")))
+#else
+#define OB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ob_status {
+  OB_OK = 0,
+  OB_ERR_NULL = 1,            /* a required pointer is NULL */
+  OB_ERR_SHAPE = 2,           /* negative size, or K / r not a multiple of 32 */
+  OB_ERR_ALIGN = 3,           /* a pointer is not 16-byte aligned */
+  OB_ERR_NAN = 4,             /* NaN in an input that must be finite */
+  OB_ERR_NOT_CONVERGED = 5,   /* SVID hit max_iters before the tolerance */
+  OB_ERR_WORKSPACE = 6,       /* workspace NULL or smaller than required */
+  OB_ERR_CUDA = 7,            /* a CUDA runtime call or kernel launch failed */
+  OB_ERR_DEVICE_TIMEOUT = 8,  /* a bounded wait inside a kernel ran out */
+  OB_ERR_UNSUPPORTED = 9,     /* device is not sm_100 or an option is unknown */
+  OB_ERR_DEVICE_BOUNDS = 10   /* a kernel's own bounds check refused an access */
+} ob_status;
+
+typedef enum ob_out_dtype {
+  OB_OUT_BF16 = 0,
+  OB_OUT_F32 = 1
+} ob_out_dtype;
+
+/* Kernel choice for ob_linear_ex / dbf_linear_ex. */
+typedef enum ob_path {
+  OB_PATH_AUTO = 0,       /* M <= decode limit: OB_PATH_TC_DECODE, else OB_PATH_TC */
+  OB_PATH_SIMT = 1,       /* CUDA-core select/add mat-vec (any M; slow for M > 4) */
+  OB_PATH_TC_DECODE = 2,  /* tcgen05, signs unpacked into tensor memory, M <= 16 per pass */
+  OB_PATH_TC = 3          /* tcgen05 tiled GEMM for large M (activations by TMA) */
+} ob_path;
+
+/* Human-readable name of a status code (static string, never NULL). */
+OB_API const char* ob_status_string(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+OB_API int ob_version(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns OB_OK, OB_ERR_DEVICE_TIMEOUT, OB_ERR_DEVICE_BOUNDS
+ * or OB_ERR_NAN (highest severity first), or OB_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+OB_API ob_status ob_last_device_error(void* stream);
+
+/*
+ * Sign extraction and packing, W_sign = Sign(W)
+ * ("1bit量化", section "rank-1 approximation": W = W_sign ⊙ |W|; the layer's
+ *  W_±1 = Sign(W) in the distillation section).
+ *   W         device, fp32 N x K, row-major; must be free of NaN.
+ *   W_packed  device, uint32 N x (K/32), written in the packed sign format.
+ * K % 32 == 0.  A NaN in W packs as +1 and sets OB_ERR_NAN in the device
+ * error word.  Asynchronous.
+ */
+OB_API ob_status ob_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* W_packed, void* stream);
+
+/* Bytes of device workspace ob_svid_rank1 needs for an N x K matrix. */
+OB_API size_t ob_svid_workspace_size(int64_t N, int64_t K);
+
+/*
+ * Rank-1 SVID of |W|: |W| ≈ a b^T with a = sqrt(sigma1) u1, b = sqrt(sigma1) v1,
+ * (u1, sigma1, v1) the leading singular triple of |W|, both vectors
+ * nonnegative ("1bit量化", section "rank-1 approximation"; the page takes the
+ * triple from an SVD, this routine finds it by power iteration on |W|^T |W|).
+ *   W          device, fp32 N x K, K % 4 == 0.
+ *   a          device, fp32 [N] (output scale, the page's h).
+ *   b          device, fp32 [K] (input scale, the page's g).
+ *   sigma1     device, fp32 [1], or NULL.
+ *   max_iters  iteration cap (<= 0 selects 200).
+ *   tol        stop when ||v_t - v_{t-1}||_2 <= tol (<= 0 selects 1e-6).
+ *   iters_out  HOST int, or NULL: iterations taken.
+ *   workspace  device, at least ob_svid_workspace_size(N, K) bytes.
+ * Synchronises `stream` once per iteration (it is an offline conversion).
+ * Returns OB_ERR_NOT_CONVERGED with the last iterate written if the cap is
+ * reached, OB_ERR_NAN if W holds NaN.  An all-zero W gives a = b = 0,
+ * sigma1 = 0 and OB_OK.
+ */
+OB_API ob_status ob_svid_rank1(const float* W, int64_t N, int64_t K,
+                        float* a, float* b, float* sigma1,
+                        int max_iters, float tol, int* iters_out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * OneBit linear layer, Proposition 1: Y = [(X ⊙ b^T) · W_sign^T] ⊙ a^T
+ * ("1bit量化", section "proposition 1").
+ *   X         device, bf16 M x K.
+ *   W_packed  device, uint32 N x (K/32), packed sign format.
+ *   a         device, fp32 [N] (the page's h).
+ *   b         device, fp32 [K] (the page's g).
+ *   Y         device, M x N, bf16 or fp32 by y_dtype.
+ * K % 32 == 0.  Accumulates in fp32.  Asynchronous.  OB_PATH_AUTO picks the
+ * tensor-memory decode kernel for M <= 16 and the tiled tcgen05 GEMM above.
+ */
+OB_API ob_status ob_linear(const void* X, int64_t M, int64_t K,
+                    const uint32_t* W_packed, int64_t N,
+                    const float* a, const float* b,
+                    void* Y, int y_dtype, void* stream);
+
+/* ob_linear with an explicit kernel choice (ob_path). */
+OB_API ob_status ob_linear_ex(const void* X, int64_t M, int64_t K,
+                       const uint32_t* W_packed, int64_t N,
+                       const float* a, const float* b,
+                       void* Y, int y_dtype, int path, void* stream);
+
+/* Bytes of device workspace dbf_linear needs (holds the M x r intermediate). */
+OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
+
+/*
+ * DBF linear layer: Y = ((((X ⊙ b^T) · S_B^T) ⊙ m^T) · S_A^T) ⊙ a^T
+ * ("Addition is almost all you need ...", section "Methodologie: Double Binary
+ *  Factorization (DBF)", inference equation).
+ *   X          device, bf16 M x K.
+ *   SB_packed  device, uint32 r x (K/32): S_B (the page's B_±1).
+ *   m          device, fp32 [r], middle scale.
+ *   SA_packed  device, uint32 N x (r/32): S_A (the page's A_±1).
+ *   a          device, fp32 [N];  b  device, fp32 [K].
+ *   Y          device, M x N, bf16 or fp32 by y_dtype.
+ *   workspace  device, at least dbf_workspace_size(M, r) bytes; holds the
+ *              intermediate T = ((X ⊙ b^T) S_B^T) ⊙ m^T between the two sign
+ *              products (it stays in L2 at the workload sizes).
+ * K % 32 == 0, r % 32 == 0.  Asynchronous.
+ */
+OB_API ob_status dbf_linear(const void* X, int64_t M, int64_t K,
+                     const uint32_t* SB_packed, int64_t r, const float* m,
+                     const uint32_t* SA_packed, int64_t N,
+                     const float* a, const float* b,
+                     void* Y, int y_dtype,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* dbf_linear with an explicit kernel choice (ob_path) for both sign products. */
+OB_API ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K,
+                        const uint32_t* SB_packed, int64_t r, const float* m,
+                        const uint32_t* SA_packed, int64_t N,
+                        const float* a, const float* b,
+                        void* Y, int y_dtype,
+                        void* workspace, size_t ws_bytes, int path, void* stream);
+
+/*
+ * Self-test of the bounded-wait machinery (no counterpart on the pages): one
+ * CTA waits on a barrier that nothing completes, gives up after `limit_ns`
+ * nanoseconds, records OB_ERR_DEVICE_TIMEOUT in the device error word and
+ * returns.  Synchronises `stream`; returns what ob_last_device_error reports
+ * (OB_ERR_DEVICE_TIMEOUT when the machinery works).
+ */
+OB_API ob_status ob_selftest_timeout(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OBGEMM_H_ */

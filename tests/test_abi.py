@@ -1,0 +1,96 @@
+"""The C-ABI library builds, loads, and exports every declared symbol (CPU only).
+
+Host-side argument checks are exercised too: they run before any CUDA call, so
+they return their status without a GPU.
+"""
+import ctypes
+import os
+
+import pytest
+
+from conftest import ROOT
+from helpers import header_functions
+
+HEADER = os.path.join(ROOT, "include", "obgemm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from binary_weight_gemm_b200 import build, _lib
+    build.build()
+    return _lib.lib()
+
+
+def test_header_declares_the_boundary():
+    names = header_functions(HEADER)
+    for required in ["ob_pack_signs", "ob_svid_rank1", "ob_linear", "dbf_linear", "ob_last_device_error",
+                     "ob_status_string", "ob_svid_workspace_size", "dbf_workspace_size"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from binary_weight_gemm_b200 import _lib
+    names = header_functions(HEADER)
+    assert names, "no declarations parsed"
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in obgemm.h but not exported"
+    assert sorted(names) == sorted(_lib.SIGNATURES), "ctypes signatures and header disagree"
+
+
+def test_library_exports_nothing_else():
+    from binary_weight_gemm_b200 import _lib
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = sorted(line.split()[-1] for line in out.splitlines() if " T " in line)
+    assert exported == sorted(_lib.SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    for code in range(11):
+        assert lib.ob_status_string(code)
+    assert b"unknown" in lib.ob_status_string(99)
+    assert lib.ob_version() >= 10000
+
+
+def test_workspace_sizes(lib):
+    assert lib.dbf_workspace_size(512, 2048) >= 512 * 2048 * 2
+    assert lib.dbf_workspace_size(0, 32) == 0
+    assert lib.ob_svid_workspace_size(4096, 4096) >= 4 * (2 * 4096 + 4096)
+    assert lib.ob_svid_workspace_size(-1, 3) == 0
+
+
+def test_host_argument_checks_without_gpu(lib):
+    OK, NULL, SHAPE, ALIGN, UNSUP = 0, 1, 2, 3, 9
+    p = ctypes.c_void_p(4096)      # never dereferenced: each check returns first
+    bad = ctypes.c_void_p(4100)    # not 16-byte aligned
+    # shapes
+    assert lib.ob_pack_signs(p, 4, 33, p, None) == SHAPE
+    assert lib.ob_pack_signs(p, -1, 32, p, None) == SHAPE
+    assert lib.ob_linear(p, 1, 48, p, 4, p, p, p, 0, None) == SHAPE
+    assert lib.dbf_linear(p, 1, 64, p, 40, p, p, 4, p, p, p, 0, p, 1 << 20, None) == SHAPE
+    # empty problems are no-ops
+    assert lib.ob_pack_signs(None, 0, 64, None, None) == OK
+    assert lib.ob_linear(None, 0, 64, None, 8, None, None, None, 0, None) == OK
+    assert lib.ob_linear(None, 3, 64, None, 0, None, None, None, 0, None) == OK
+    # options
+    assert lib.ob_linear(p, 1, 64, p, 4, p, p, p, 7, None) == UNSUP
+    assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, 42, None) == UNSUP
+    # null and alignment
+    assert lib.ob_linear(None, 1, 64, p, 4, p, p, p, 0, None) == NULL
+    assert lib.ob_linear(p, 1, 64, p, 4, p, p, None, 0, None) == NULL
+    assert lib.ob_linear(bad, 1, 64, p, 4, p, p, p, 0, None) == ALIGN
+    assert lib.ob_pack_signs(bad, 2, 64, p, None) == ALIGN
+    assert lib.dbf_linear(p, 1, 64, p, 32, p, p, 4, p, p, p, 0, None, 0, None) == 6  # workspace
+    assert lib.dbf_linear(p, 1, 64, p, 32, None, p, 4, p, p, p, 0, p, 1 << 20, None) == NULL
+    iters = ctypes.c_int(-1)
+    assert lib.ob_svid_rank1(p, 4, 64, p, p, None, 0, 0.0, ctypes.byref(iters), None, 0, None) == 6
+    assert iters.value == 0
+    assert lib.ob_svid_rank1(p, 4, 62, p, p, None, 0, 0.0, None, p, 1 << 20, None) == SHAPE
+
+
+def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from binary_weight_gemm_b200 import _lib
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_LIB", None)
+    with pytest.raises(ImportError):
+        _lib.lib()

@@ -1,0 +1,86 @@
+"""GPU parity of the DBF linear layer against the fp64 oracle (direct form W_hat = diag(a) S_A diag(m) S_B diag(b))."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from binary_weight_gemm_b200 import synth
+from helpers import assert_gemm_close
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"simt": 1, "tc_decode": 2, "tc": 3, "auto": 0}
+
+
+@pytest.fixture(scope="module")
+def ops():
+    from binary_weight_gemm_b200 import build
+    build.build()
+    from binary_weight_gemm_b200 import ops as _ops
+    torch.cuda.init()
+    return _ops
+
+
+def _cuda(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _run(ops, xb, f, path, out_dtype=torch.bfloat16):
+    SB = ops.ob_pack_signs(_cuda(f["S_B"].astype(np.float32)))
+    SA = ops.ob_pack_signs(_cuda(f["S_A"].astype(np.float32)))
+    X = _cuda(xb.view(np.int16)).view(torch.bfloat16)
+    Y = ops.dbf_linear(X, SB, _cuda(f["m"]), SA, _cuda(f["a"]), _cuda(f["b"]), out_dtype=out_dtype, path=path)
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    return Y
+
+
+def _ref(x, f):
+    return oracle.dbf_linear(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"])
+
+
+@pytest.mark.parametrize("path", ["simt", "tc_decode", "tc"])
+@pytest.mark.parametrize("M,N,r,K", [(1, 128, 32, 64), (4, 256, 96, 256), (7, 200, 160, 96), (33, 130, 64, 128),
+                                     (260, 256, 128, 320)])
+def test_dbf_small_shapes(ops, path, M, N, r, K):
+    f = synth.dbf_factors(M + N + r + K, N, r, K)
+    xb, x = synth.activations(M + N, M, K)
+    assert_gemm_close(_run(ops, xb, f, PATHS[path]), _ref(x, f), what=f"dbf {path} {M},{N},{r},{K}")
+
+
+@pytest.mark.parametrize("M", [1, 512])
+def test_dbf_workload_full(ops, M):
+    # DBF: K = N = 4096, r = 2048; S_A, S_B random +/-1; a, m, b ~ |N(0,1)|*0.02+1e-3.
+    f = synth.dbf_factors(3, 4096, 2048, 4096)
+    xb, x = synth.activations(3, M, 4096)
+    Y = _run(ops, xb, f, PATHS["auto"])
+    assert_gemm_close(Y, _ref(x, f), what=f"dbf workload M={M}")
+
+
+def test_dbf_fp32_output(ops):
+    # Smallest middle dimension (one packed word per S_A row), fp32 output.
+    f = synth.dbf_factors(11, 256, 32, 256)
+    xb, x = synth.activations(11, 3, 256)
+    Y = _run(ops, xb, f, PATHS["auto"], out_dtype=torch.float32)
+    assert Y.dtype == torch.float32
+    assert_gemm_close(Y, _ref(x, f), what="dbf fp32")
+
+
+def test_dbf_one_hot_input(ops):
+    f = synth.dbf_factors(12, 128, 64, 128)
+    ks = [0, 5, 31, 32, 127]
+    x = np.zeros((len(ks), 128), dtype=np.float32)
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    xb, x = synth.bf16_round(x)
+    Y = _run(ops, xb, f, PATHS["auto"], out_dtype=torch.float32)
+    assert_gemm_close(Y, _ref(x, f), what="dbf one-hot")
+
+
+def test_dbf_degenerate(ops):
+    f = synth.dbf_factors(13, 64, 32, 64)
+    X = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    SB = ops.ob_pack_signs(_cuda(f["S_B"].astype(np.float32)))
+    SA = ops.ob_pack_signs(_cuda(f["S_A"].astype(np.float32)))
+    Y = ops.dbf_linear(X, SB, _cuda(f["m"]), SA, _cuda(f["a"]), _cuda(f["b"]))
+    assert Y.shape == (0, 64)

@@ -1,0 +1,205 @@
+"""GPU parity of the OneBit linear layer against the fp64 oracle (direct form).
+
+Tolerances (bf16 inputs, fp32 accumulation): relative Frobenius error <= 5e-3 and
+max |dY| <= 1e-2 * max |Y_ref|.  a, b are the oracle's SVID vectors cast to
+fp32 and given to both sides, so the GEMM is tested in isolation; one test runs
+the whole GPU pipeline (pack, SVID, linear) against the whole oracle pipeline.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from binary_weight_gemm_b200 import synth
+from helpers import assert_gemm_close, oracle_svid
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"simt": 1, "tc_decode": 2, "tc": 3}
+
+
+@pytest.fixture(scope="module")
+def ops():
+    from binary_weight_gemm_b200 import build
+    build.build()
+    from binary_weight_gemm_b200 import ops as _ops
+    torch.cuda.init()
+    return _ops
+
+
+def _cuda(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _x_bf16(x_bits):
+    return _cuda(x_bits.view(np.int16)).view(torch.bfloat16)
+
+
+def _run(ops, x_bits, W, a, b, path, out_dtype=torch.bfloat16):
+    P = ops.ob_pack_signs(_cuda(W))
+    Y = ops.ob_linear(_x_bf16(x_bits), P, _cuda(a), _cuda(b), out_dtype=out_dtype, path=path)
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    return Y
+
+
+def _ref(x, W, a, b):
+    return oracle.onebit_linear(x, oracle.sign_pm1(W), a, b)
+
+
+# ---------------------------------------------------------------- small and ragged shapes, every path
+
+SHAPES = [  # (M, N, K)
+    (4, 256, 256),     # the tiny workload
+    (1, 128, 64),
+    (3, 200, 96),      # ragged N (not a multiple of 128), K with a half 64-stage
+    (5, 129, 32),      # one packed word per row
+    (16, 384, 1024),
+    (17, 130, 160),    # M over one decode pass
+    (300, 260, 192),   # ragged M and N tiles for the large-M kernel
+    (513, 128, 4096),
+]
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_linear_small_shapes(ops, path, M, N, K):
+    seed = M * 7 + N + K
+    W = synth.weights(seed, N, K)
+    a, b, _ = oracle.svid_rank1(W)
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    xb, x = synth.activations(seed, M, K)
+    Y = _run(ops, xb, W, a, b, PATHS[path])
+    assert_gemm_close(Y, _ref(x, W, a, b), what=f"{path} {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_linear_one_hot_rows_pin_layout(ops, path):
+    # X = e_k picks column k of W_hat: Y[:, n] = a_n s_nk b_k.  Pins bit order and orientation.
+    N, K = 256, 256
+    W = synth.weights(21, N, K)
+    a, b, _ = oracle.svid_rank1(W)
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    ks = [0, 1, 15, 16, 17, 31, 32, 63, 64, 100, 255]
+    x = np.zeros((len(ks), K), dtype=np.float32)
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    xb, x = synth.bf16_round(x)
+    Y = _run(ops, xb, W, a, b, PATHS[path], out_dtype=torch.float32).cpu().numpy()
+    ref = _ref(x, W, a, b)
+    np.testing.assert_allclose(Y, ref, rtol=1e-2, atol=1e-7)
+    assert np.array_equal(np.sign(Y), np.sign(ref))
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_linear_fp32_output_and_outliers(ops, path):
+    M, N, K = 8, 384, 512
+    W = synth.weights(31, N, K)
+    a, b, _ = oracle.svid_rank1(W)
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    xb, x = synth.activations(31, M, K, outliers=True)
+    Y = _run(ops, xb, W, a, b, PATHS[path], out_dtype=torch.float32)
+    assert Y.dtype == torch.float32
+    assert_gemm_close(Y, _ref(x, W, a, b), what=path)
+
+
+def test_linear_exact_rank1_pipeline(ops):
+    # |W| rank 1: GPU SVID is exact and the OneBit layer reproduces the dense X W^T.
+    rng = np.random.default_rng(5)
+    N, K, M = 256, 512, 4
+    p = rng.uniform(0.5, 2.0, N).astype(np.float32) * 0.02
+    q = rng.uniform(0.5, 2.0, K).astype(np.float32)
+    W = (np.where(rng.random((N, K)) < 0.5, -1, 1) * np.outer(p, q)).astype(np.float32)
+    xb, x = synth.activations(5, M, K)
+    a, b, _, _, st = ops.ob_svid_rank1(_cuda(W))
+    P = ops.ob_pack_signs(_cuda(W))
+    for path in PATHS.values():
+        Y = ops.ob_linear(_x_bf16(xb), P, a, b, out_dtype=torch.float32, path=path)
+        assert_gemm_close(Y, x.astype(np.float64) @ W.astype(np.float64).T, what=f"path {path}")
+
+
+def test_linear_end_to_end_pipeline_vs_oracle_pipeline(ops):
+    # GPU: pack + SVID + linear.  Oracle: Sign + full-SVD SVID + direct form.
+    W = synth.weights(0, 256, 256)
+    xb, x = synth.activations(0, 4, 256)
+    a_g, b_g, _, _, _ = ops.ob_svid_rank1(_cuda(W))
+    P = ops.ob_pack_signs(_cuda(W))
+    a_r, b_r, _ = oracle.svid_rank1(W)
+    ref = oracle.onebit_linear(x, oracle.sign_pm1(W), a_r, b_r)
+    for path in PATHS.values():
+        Y = ops.ob_linear(_x_bf16(xb), P, a_g, b_g, path=path)
+        assert_gemm_close(Y, ref, what=f"pipeline path {path}")
+
+
+def test_linear_degenerate_sizes(ops):
+    P = torch.zeros((8, 2), dtype=torch.int32, device="cuda")
+    a = torch.ones(8, device="cuda")
+    b = torch.ones(64, device="cuda")
+    Y = ops.ob_linear(torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda"), P, a, b)
+    assert Y.shape == (0, 8)
+    # K = 0: empty sum, Y = 0.
+    Y = ops.ob_linear(torch.zeros((3, 0), dtype=torch.bfloat16, device="cuda"),
+                      torch.zeros((8, 0), dtype=torch.int32, device="cuda"), a,
+                      torch.ones(0, device="cuda"), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert Y.shape == (3, 8) and not Y.any()
+
+
+# ---------------------------------------------------------------- full-size workloads
+
+@pytest.mark.parametrize("path", ["tc_decode", "simt"])
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_workload_full(ops, path, M):
+    # OneBit decode GEMV: X M x 4096, W 4096 x 4096 -> 2 MiB packed, a, b from SVID.
+    W, a, b, _ = oracle_svid(1, 4096, 4096)
+    xb, x = synth.activations(1, M, 4096)
+    Y = _run(ops, xb, W, a, b, PATHS[path])
+    assert_gemm_close(Y, _ref(x, W, a, b), what=f"decode M={M} {path}")
+
+
+def test_prefill_workload_full_sampled_rows(ops):
+    # OneBit prefill: X 2048 x 4096, W 11008 x 4096; oracle on 64 sampled token rows.
+    W, a, b, _ = oracle_svid(2, 11008, 4096)
+    xb, x = synth.activations(2, 2048, 4096)
+    Y = _run(ops, xb, W, a, b, PATHS["tc"])
+    rows = np.random.default_rng(0).choice(2048, 64, replace=False)
+    rows[:2] = [0, 2047]
+    assert_gemm_close(Y[torch.from_numpy(rows).cuda()], _ref(x[rows], W, a, b), what="prefill rows")
+    assert torch.isfinite(Y.float()).all()
+
+
+SWEEP = [(4096, 4096), (4096, 11008), (11008, 4096)]  # (K, N): K -> N
+
+
+@pytest.mark.parametrize("shape_idx", range(3))
+@pytest.mark.parametrize("M", [1, 16, 256, 4096])
+def test_sweep_with_outliers(ops, shape_idx, M):
+    K, N = SWEEP[shape_idx]
+    W, a, b, _ = oracle_svid(4 + shape_idx, N, K)
+    xb, x = synth.activations(4 + shape_idx, M, K, outliers=True)
+    Y = _run(ops, xb, W, a, b, 0)
+    if M <= 256:
+        assert_gemm_close(Y, _ref(x, W, a, b), what=f"sweep {K}->{N} M={M}")
+    else:
+        rows = np.random.default_rng(1).choice(M, 32, replace=False)
+        rows[:2] = [0, M - 1]
+        assert_gemm_close(Y[torch.from_numpy(rows).cuda()], _ref(x[rows], W, a, b), what=f"sweep rows M={M}")
+
+
+def test_cuda_graph_replay_matches(ops):
+    W, a, b, _ = oracle_svid(1, 4096, 4096)
+    xb, x = synth.activations(1, 4, 4096)
+    P = ops.ob_pack_signs(_cuda(W))
+    X, A, B = _x_bf16(xb), _cuda(a), _cuda(b)
+    Y = torch.empty((4, 4096), dtype=torch.bfloat16, device="cuda")
+    ops.ob_linear(X, P, A, B, out=Y)  # warm up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            ops.ob_linear(X, P, A, B, out=Y, stream=s)
+    Y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert_gemm_close(Y, _ref(x, W, a, b), what="graph replay")
