@@ -4,16 +4,18 @@
 // "Addition is almost all you need ..." (gist.science), "Methodologie": products
 // with +/-1 matrices become additions and subtractions.
 //
-// Each warp owns rows of S; lane l streams 128-bit groups of four packed words
-// (group index c = l + 32 j), so a warp load covers 512 contiguous bytes.  The
-// pre-scaled activations x' = x ⊙ b live in shared memory as fp32 in a layout
-// where lane l always reads bank (const + l): element (token m, bit i, word q of
-// group c) sits at ((m*32 + i)*Q + q) * pitch + c.  Sign bit i of a word is
-// moved to bit 31 and XORed into x' before the add, so no multiply touches a
-// sign.  Lane partial sums are reduced with warp shuffles; the output scale a
-// and the store are fused.  Handles MT <= 4 tokens per pass (the host loops
-// over token groups); it is the baseline the tensor-core decode kernel is
-// measured against.
+// Each warp owns kRowsPerWarp rows of S.  K is processed in chunks of 32 lane
+// groups; lane l owns group l of the chunk, i.e. Q consecutive packed words
+// loaded with one 128-bit (Q = 4) or 32-bit (Q = 1) load, so a warp load covers
+// 512 (or 128) contiguous bytes.  The pre-scaled activations x' = x ⊙ b live in
+// shared memory as fp32 in a layout where lane l always reads bank (const + l):
+// element (token m, bit i, word q of group c) sits at ((m*32 + i)*Q + q) * 33 + c.
+// Sign bit i of a word is moved to bit 31 and XORed into x' before the add, so no
+// multiply touches a sign.  Lane partial sums are reduced with warp shuffles; the
+// output scale a and the store are fused.  At decode sizes the kernel is
+// latency-bound, so every global load of a chunk (the warp's sign words, then
+// the activations and scales it stages) is issued before any of them is used.
+// Handles MT <= 4 tokens per pass (the host loops over token groups).
 #include "ob_device.cuh"
 #include "ob_internal.h"
 
@@ -22,23 +24,23 @@ namespace {
 
 constexpr int kSimtThreads = 256;
 constexpr int kSimtWarps = kSimtThreads / 32;
-constexpr int kRowsPerWarp = 2;
-constexpr int kRowsPerCta = kSimtWarps * kRowsPerWarp;
-constexpr int kStageFloats = 24576;  // ~96 KB of staged x' per chunk
-
-// Groups (of Q words) staged per chunk so that MT x 32 x Q x pitch floats fit the stage.
-template <int MT, int Q>
-__host__ __device__ constexpr int groups_per_chunk() { return kStageFloats / (MT * 32 * Q) - 1; }
+// Rows per warp shrink as tokens per pass grow, to keep the accumulators in registers.
+template <int MT>
+__host__ __device__ constexpr int rows_per_warp() { return MT >= 4 ? 1 : (MT == 2 ? 2 : 4); }
+constexpr int kPitch = 33;  // 32 groups + 1: odd pitch
 
 template <int MT, int Q>
 __global__ void __launch_bounds__(kSimtThreads) sign_gemv_simt_kernel(SignGemmArgs g, int64_t m0) {
-  extern __shared__ float xs[];
+  constexpr int kRowsPerWarp = rows_per_warp<MT>();
+  constexpr int kRowsPerCta = kSimtWarps * kRowsPerWarp;
+  extern __shared__ float xs[];  // [MT][32][Q][kPitch]
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t K = g.K;
-  const int64_t Wd = K / 32;           // words per row
-  const int64_t G = Wd / Q;            // groups per row
+  const int64_t Wd = K / 32;              // words per row
+  const int64_t G = (Wd + Q - 1) / Q;     // groups per row (Q = 4 only when Wd % 4 == 0)
   const int64_t mt = min64(MT, g.M - m0);
+  const int64_t row0 = (int64_t)blockIdx.x * kRowsPerCta + warp * kRowsPerWarp;
 
   float acc[kRowsPerWarp][MT];
 #pragma unroll
@@ -46,59 +48,84 @@ __global__ void __launch_bounds__(kSimtThreads) sign_gemv_simt_kernel(SignGemmAr
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
 
-  const int64_t row0 = (int64_t)blockIdx.x * kRowsPerCta + warp * kRowsPerWarp;
-
-  constexpr int kChunk = groups_per_chunk<MT, Q>();
-  for (int64_t c0 = 0; c0 < G; c0 += kChunk) {
-    const int cg = (int)min64(kChunk, G - c0);
-    const int pitch = cg | 1;  // odd pitch: conflict-free staging stores
-    __syncthreads();
-    // Stage x'[m][k] for k in [32*Q*c0, 32*Q*(c0+cg)).
-    const int total = MT * 32 * Q * cg;
-    for (int idx = threadIdx.x; idx < total; idx += kSimtThreads) {
-      const int m = idx / (32 * Q * cg);
-      const int rem = idx - m * (32 * Q * cg);
-      const int w_local = rem >> 5;       // word within chunk
-      const int i = rem & 31;             // bit
-      const int c = w_local / Q, q = w_local - c * Q;
-      const int64_t k = (c0 * Q + w_local) * 32 + i;
-      float v = 0.f;
-      if (m < mt) {
-        v = bf16_bits_to_float(g.X[(m0 + m) * K + k]);
-        if (g.iscale) v *= __ldg(g.iscale + k);
-      }
-      xs[((m * 32 + i) * Q + q) * pitch + c] = v;
-    }
-    __syncthreads();
+  constexpr int kChunkK = 32 * Q * 32;                 // k per chunk: 32 groups of Q words
+  constexpr int kPerThread = kChunkK / kSimtThreads;   // staged k per thread (16 or 4)
+  for (int64_t c0 = 0; c0 < G; c0 += 32) {
+    // 1. This lane's sign words for every row of the warp (independent loads).
+    uint32_t wq[kRowsPerWarp][Q];
+    const int64_t grp = c0 + lane;
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r) {
       const int64_t n = row0 + r;
-      if (n >= g.R) break;
-      const uint32_t* srow = g.S + n * Wd + c0 * Q;
-      for (int c = lane; c < cg; c += 32) {
-        uint32_t wq[Q];
-        if constexpr (Q == 4) {
-          const uint4 v = __ldcs(reinterpret_cast<const uint4*>(srow) + c);
-          wq[0] = v.x; wq[1] = v.y; wq[2] = v.z; wq[3] = v.w;
-        } else {
-          wq[0] = __ldcs(srow + c);
+      const bool ok = n < g.R && grp < G;
+      const uint32_t* srow = g.S + (ok ? n : 0) * Wd;
+      if constexpr (Q == 4) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (ok) v = __ldcs(reinterpret_cast<const uint4*>(srow) + grp);
+        wq[r][0] = v.x; wq[r][1] = v.y; wq[r][2] = v.z; wq[r][3] = v.w;
+      } else {
+        wq[r][0] = ok ? __ldcs(srow + grp) : 0u;
+      }
+    }
+    // 2. Stage x' for this chunk: thread t owns kPerThread consecutive k for all tokens.
+    {
+      const int64_t kb = c0 * Q * 32 + (int64_t)threadIdx.x * kPerThread;
+      float sc[kPerThread];
+      uint32_t xv[MT][kPerThread / 2];  // bf16 pairs, as loaded
+#pragma unroll
+      for (int e = 0; e < kPerThread; e += 4) {
+        float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (kb + e < K) s4 = g.iscale ? __ldg(reinterpret_cast<const float4*>(g.iscale + kb + e))
+                                      : make_float4(1.f, 1.f, 1.f, 1.f);
+        sc[e] = s4.x; sc[e + 1] = s4.y; sc[e + 2] = s4.z; sc[e + 3] = s4.w;
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+#pragma unroll
+        for (int e = 0; e < kPerThread; e += 4) {
+          uint2 v = make_uint2(0u, 0u);
+          if (m < mt && kb + e < K) v = __ldg(reinterpret_cast<const uint2*>(g.X + (m0 + m) * K + kb + e));
+          xv[m][e / 2] = v.x;
+          xv[m][e / 2 + 1] = v.y;
         }
+      }
+      __syncthreads();  // previous chunk's readers are done with xs
 #pragma unroll
-        for (int q = 0; q < Q; ++q) {
+      for (int e = 0; e < kPerThread; ++e) {
+        const int kl = threadIdx.x * kPerThread + e;  // k within the chunk
+        const int w_local = kl >> 5, i = kl & 31;
+        const int c = w_local / Q, q = w_local % Q;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint32_t sbit = (wq[q] << (31 - i)) & 0x80000000u;
+        for (int m = 0; m < MT; ++m) {
+          const uint32_t pr = xv[m][e / 2];
+          const float x = __uint_as_float((e & 1) ? (pr & 0xFFFF0000u) : (pr << 16));
+          xs[((m * 32 + i) * Q + q) * kPitch + c] = x * sc[e];
+        }
+      }
+      __syncthreads();
+    }
+    // 3. Select/add: sign bit i of each word XORed into x'.
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              const float x = xs[((m * 32 + i) * Q + q) * pitch + c];
-              acc[r][m] += __uint_as_float(__float_as_uint(x) ^ sbit);
-            }
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const uint32_t sbit = (wq[r][q] << (31 - i)) & 0x80000000u;
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const float x = xs[((m * 32 + i) * Q + q) * kPitch + lane];
+            acc[r][m] += __uint_as_float(__float_as_uint(x) ^ sbit);
           }
         }
       }
     }
   }
 
+  // 4. Warp reduction, output scale, store.
+  float osc[kRowsPerWarp];
+#pragma unroll
+  for (int r = 0; r < kRowsPerWarp; ++r) osc[r] = (row0 + r < g.R) ? __ldg(g.oscale + row0 + r) : 0.f;
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) {
     const int64_t n = row0 + r;
@@ -114,7 +141,7 @@ __global__ void __launch_bounds__(kSimtThreads) sign_gemv_simt_kernel(SignGemmAr
 #pragma unroll
       for (int m = 0; m < MT; ++m)
         if (m == lane) v = acc[r][m];
-      v *= __ldg(g.oscale + n);
+      v *= osc[r];
       const int64_t off = (m0 + lane) * g.ldy + n;
       if (g.y_dtype == OB_OUT_F32)
         static_cast<float*>(g.Y)[off] = v;
@@ -126,14 +153,13 @@ __global__ void __launch_bounds__(kSimtThreads) sign_gemv_simt_kernel(SignGemmAr
 
 template <int MT, int Q>
 cudaError_t launch_one(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c) {
-  const int64_t G = g.K / 32 / Q;
-  const int cg = (int)std::min<int64_t>(groups_per_chunk<MT, Q>(), G);
-  const size_t smem = sizeof(float) * (size_t)MT * 32 * Q * (size_t)(cg | 1);
+  const size_t smem = sizeof(float) * (size_t)MT * 32 * Q * kPitch;
   auto kern = sign_gemv_simt_kernel<MT, Q>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
+  constexpr int kRowsPerCta = kSimtWarps * rows_per_warp<MT>();
   const unsigned blocks = (unsigned)((g.R + kRowsPerCta - 1) / kRowsPerCta);
   kern<<<blocks, kSimtThreads, smem, c.stream>>>(g, m0);
   return cudaGetLastError();

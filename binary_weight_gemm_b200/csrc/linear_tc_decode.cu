@@ -18,13 +18,22 @@
 //    the same (i, i+16) pairing order so the MMA contracts matching k.
 //  * One elected thread issues tcgen05.mma (M=128, N=16, K=16, fp32 accumulate
 //    in TMEM) per 16 k; A stages cycle through a ring of TMEM slots guarded by
-//    mbarriers (threads -> full, tcgen05.commit -> empty).
+//    mbarriers (threads -> full, tcgen05.commit -> empty).  An N=16 MMA is
+//    short, so a chain of MMAs into one accumulator runs at the MMA latency,
+//    not its throughput: k sub-step q of every stage goes to its own
+//    accumulator D_q, four independent chains summed in the epilogue.
 //  * K is split over the CTAs of a thread-block cluster; the partial 128 x 16
 //    tiles are reduced through distributed shared memory, scaled by oscale and
 //    stored (bf16 or fp32).  No global workspace and no atomics.
-//  * Weight words are requested before the programmatic-dependent-launch wait
-//    and the first ring of sign stages is expanded before it too: only the
-//    activations depend on the previous kernel in the stream.
+//  * The kernel is latency-bound at decode sizes, so every global load is
+//    issued as early as it can be: all of a CTA's packed words go to registers
+//    at kernel start, and the first ring of sign stages is expanded into TMEM,
+//    before the programmatic-dependent-launch wait -- only the activations
+//    depend on the previous kernel in the stream.  The activation loads are
+//    all issued before any of them is used.  Weight loads are issued before
+//    the TMEM allocation.  Each CTA allocates 256 of the SM's 512 TMEM columns,
+//    so two CTAs (of this call or the next) always fit side by side and no
+//    allocation can wait on a CTA of its own cluster.
 #include <algorithm>
 #include <cstdlib>
 
@@ -37,10 +46,13 @@ namespace {
 constexpr int kRows = 128;          // weight rows per CTA (MMA M)
 constexpr int kTok = 16;            // tokens per pass (MMA N)
 constexpr int kStageK = 64;         // k per stage (one 128-byte swizzle row of bf16)
-constexpr int kRing = 6;            // TMEM A-slots
-constexpr int kTmemCols = 256;      // D at columns [0,16), A slots at 32 + 32*s
-constexpr int kMaxStagesPerCta = 48;
-constexpr int kThreads = 160;       // warps 0-3: rows (unpack, X' prep, epilogue); warp 4: TMEM + MMA
+constexpr int kAcc = 4;             // independent accumulators: D_q at columns 16q, q < 4
+constexpr int kRingBase = 16 * kAcc;
+constexpr int kRing = 6;            // TMEM A-slots: columns kRingBase + 32*s, s < 6
+constexpr int kTmemCols = 256;      // two CTAs per SM always fit
+constexpr int kMaxStagesPerCta = 32;
+constexpr int kMaxWords = 2 * kMaxStagesPerCta;
+constexpr int kThreads = 160;       // warps 0-3: rows (expand, X' staging, epilogue); warp 4: TMEM + MMA
 constexpr uint32_t kAtomBytes = kTok * 128;  // one stage of X': 16 rows x 128 B
 constexpr uint32_t kIdesc = idesc_bf16_f32(kRows, kTok);
 
@@ -80,10 +92,17 @@ __device__ __forceinline__ void expand_stage(uint32_t w0, uint32_t w1, uint32_t 
   }
 }
 
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned* err, volatile int* abort_flag,
+                                          int lane) {
+  int okw = 1;
+  if (lane == 0) okw = mbar_wait(bar, parity, err, abort_flag) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, okw, 0) != 0;
+}
+
 template <bool kCluster>
-__global__ void __launch_bounds__(kThreads) sign_gemm_tc_decode_kernel(SignGemmArgs g, int64_t m0,
-                                                                        int stages_total, int ksplit,
-                                                                        unsigned* err) {
+__global__ void __launch_bounds__(kThreads, 2) sign_gemm_tc_decode_kernel(SignGemmArgs g, int64_t m0,
+                                                                           int stages_total, int ksplit,
+                                                                           unsigned* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // X' atoms first (1024-byte aligned for the swizzle), then the control block.
   uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -99,6 +118,29 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_tc_decode_kernel(SignGemmA
   const int64_t Wd = K / 32;
   const int64_t n0 = (int64_t)blockIdx.y * kRows;
   const int64_t mt = min64(kTok, g.M - m0);
+
+  // Row threads request their packed words first: they depend on nothing.
+  const int64_t n = n0 + (tid & 127);
+  const bool row_ok = warp < 4 && n < g.R;
+  const int64_t w_begin = (int64_t)st0 * 2;  // even
+  const int nw = (int)(min64(Wd, (int64_t)st1 * 2) - w_begin);
+  // All of this row's words for the CTA's k range, requested at once.
+  uint32_t w[kMaxWords];
+  if ((Wd & 1) == 0) {  // rows and w_begin are 8-byte aligned: two words per load
+    const uint2* src = reinterpret_cast<const uint2*>(g.S + (row_ok ? n : 0) * Wd + w_begin);
+#pragma unroll
+    for (int i = 0; i < kMaxWords / 2; ++i) {
+      uint2 v = make_uint2(0u, 0u);
+      if (row_ok && 2 * i < nw) v = __ldg(src + i);
+      w[2 * i] = v.x;
+      w[2 * i + 1] = v.y;
+    }
+  } else {
+    const uint32_t* src = g.S + (row_ok ? n : 0) * Wd + w_begin;
+#pragma unroll
+    for (int i = 0; i < kMaxWords; ++i) w[i] = (row_ok && i < nw) ? __ldg(src + i) : 0u;
+  }
+  const float osc = row_ok ? __ldg(g.oscale + n) : 0.f;
 
   if (tid == 0) {
     for (int s = 0; s < kRing; ++s) {
@@ -124,56 +166,32 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_tc_decode_kernel(SignGemmA
   if (warp < 4) {
     // ------------------------------------------------ row threads
     const int t = tid;                      // row within the tile == TMEM lane
-    const int64_t n = n0 + t;
-    const bool row_ok = n < g.R;
-    const uint32_t* srow = g.S + (row_ok ? n : 0) * Wd;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const int64_t w_begin = (int64_t)st0 * 2;
-    const int64_t w_end = min64(Wd, (int64_t)st1 * 2);
 
-    // Words of ring round r (stages r*kRing .. r*kRing+kRing-1) of this row.
-    auto load_round = [&](uint32_t (&buf)[2 * kRing], int r) {
+
+    // First ring round: every slot is free.
 #pragma unroll
-      for (int i = 0; i < 2 * kRing; ++i) {
-        const int64_t w = w_begin + (int64_t)r * 2 * kRing + i;
-        buf[i] = (row_ok && w < w_end) ? __ldg(srow + w) : 0u;
-      }
-    };
-    // Expand round r into the ring (round 0 finds every slot free).
-    auto process_round = [&](const uint32_t (&buf)[2 * kRing], int r) -> bool {
-#pragma unroll
-      for (int jj = 0; jj < kRing; ++jj) {
-        const int j = r * kRing + jj;
-        if (j >= nst) break;
+    for (int j = 0; j < kRing; ++j) {
+      if (j < nst) {
         uint32_t v[32];
-        expand_stage(buf[2 * jj], buf[2 * jj + 1], v);
-        if (r > 0) {
-          int okw = 1;
-          if (lane == 0) okw = mbar_wait(&sh->empty[jj], (uint32_t)(r - 1) & 1u, err, abort_flag) ? 1 : 0;
-          if (!__shfl_sync(0xffffffffu, okw, 0)) return false;
-          tc_fence_after();
-        }
-        tmem_st_x32(lane_base + 32u + 32u * jj, v);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->full[jj]);
+        expand_stage(w[2 * j], w[2 * j + 1], v);
+        tmem_st_x32(lane_base + kRingBase + 32u * j, v);
       }
-      return true;
-    };
-
-    // Weight words do not depend on the previous grid: request two rounds and
-    // expand the first before the dependency wait.
-    uint32_t wa[2 * kRing], wb[2 * kRing];
-    load_round(wa, 0);
-    load_round(wb, 1);
-    bool ok = process_round(wa, 0);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < kRing; ++j)
+        if (j < nst) mbar_arrive(&sh->full[j]);
+    }
 
     // Activations depend on the previous grid in the stream.
     pdl_wait();
 
     // X' = x ⊙ iscale into the swizzled B tile, in (i, i+16) pair order.
-    // Unit = (token half h, stage j, word g, 8-column block cb): 8 pairs -> 32 bytes.
+    // Unit = (token half h, stage j, word g, 8-column block cb): 8 tokens x 8 pairs.
     {
       const int units = 2 * nst * 4;
       for (int u = t; u < units; u += 128) {
@@ -184,25 +202,38 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_tc_decode_kernel(SignGemmA
         const int cb = rest & 1;
         const int64_t k_lo = (int64_t)(st0 + j) * kStageK + gw * 32 + cb * 8;  // 8 consecutive k
         const int64_t k_hi = k_lo + 16;
+        const bool blk_ok = k_lo < K;  // K % 32 == 0: the whole (k_lo, k_hi) block is in or out
         float slo[8], shi[8];
-        const bool lo_ok = k_lo < K, hi_ok = k_hi < K;  // K % 32 == 0: blocks are all-in or all-out
+        if (g.iscale && blk_ok) {
+          const float4* s4 = reinterpret_cast<const float4*>(g.iscale + k_lo);
+          const float4 a0 = __ldg(s4), a1 = __ldg(s4 + 1), b0 = __ldg(s4 + 4), b1 = __ldg(s4 + 5);
+          slo[0] = a0.x; slo[1] = a0.y; slo[2] = a0.z; slo[3] = a0.w;
+          slo[4] = a1.x; slo[5] = a1.y; slo[6] = a1.z; slo[7] = a1.w;
+          shi[0] = b0.x; shi[1] = b0.y; shi[2] = b0.z; shi[3] = b0.w;
+          shi[4] = b1.x; shi[5] = b1.y; shi[6] = b1.z; shi[7] = b1.w;
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          slo[e] = (g.iscale && lo_ok) ? __ldg(g.iscale + k_lo + e) : 1.f;
-          shi[e] = (g.iscale && hi_ok) ? __ldg(g.iscale + k_hi + e) : 1.f;
+          for (int e = 0; e < 8; ++e) slo[e] = shi[e] = 1.f;
         }
-        uint8_t* atom = xs + (size_t)j * kAtomBytes;
-#pragma unroll 2
+        uint4 xlo[8], xhi[8];
+#pragma unroll
         for (int mm = 0; mm < 8; ++mm) {
           const int m = h * 8 + mm;
-          uint4 xlo = make_uint4(0, 0, 0, 0), xhi = make_uint4(0, 0, 0, 0);
-          if (m < mt) {
+          xlo[mm] = make_uint4(0, 0, 0, 0);
+          xhi[mm] = make_uint4(0, 0, 0, 0);
+          if (m < mt && blk_ok) {
             const uint16_t* xrow = g.X + (m0 + m) * K;
-            if (lo_ok) xlo = __ldg(reinterpret_cast<const uint4*>(xrow + k_lo));
-            if (hi_ok) xhi = __ldg(reinterpret_cast<const uint4*>(xrow + k_hi));
+            xlo[mm] = __ldg(reinterpret_cast<const uint4*>(xrow + k_lo));
+            xhi[mm] = __ldg(reinterpret_cast<const uint4*>(xrow + k_hi));
           }
-          const uint32_t lo_w[4] = {xlo.x, xlo.y, xlo.z, xlo.w};
-          const uint32_t hi_w[4] = {xhi.x, xhi.y, xhi.z, xhi.w};
+        }
+        uint8_t* atom = xs + (size_t)j * kAtomBytes;
+        const uint32_t e0 = (uint32_t)(gw * 32 + cb * 16);  // element index of pair (gw*16 + cb*8)
+#pragma unroll
+        for (int mm = 0; mm < 8; ++mm) {
+          const int m = h * 8 + mm;
+          const uint32_t lo_w[4] = {xlo[mm].x, xlo[mm].y, xlo[mm].z, xlo[mm].w};
+          const uint32_t hi_w[4] = {xhi[mm].x, xhi[mm].y, xhi[mm].z, xhi[mm].w};
           uint32_t out[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -211,8 +242,6 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_tc_decode_kernel(SignGemmA
             const float xh = __uint_as_float((e & 1) ? (hw & 0xFFFF0000u) : (hw << 16)) * shi[e];
             out[e] = pack_bf16x2(xl, xh);
           }
-          // Pair index within the stage row: gw*16 + cb*8 + e -> element 2*(that).
-          const uint32_t e0 = (uint32_t)(gw * 32 + cb * 16);
           *reinterpret_cast<uint4*>(atom + sw128_offset(m, e0)) = make_uint4(out[0], out[1], out[2], out[3]);
           *reinterpret_cast<uint4*>(atom + sw128_offset(m, e0 + 8)) = make_uint4(out[4], out[5], out[6], out[7]);
         }
@@ -222,41 +251,52 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_tc_decode_kernel(SignGemmA
       if (t == 0) mbar_arrive(&sh->xready);
     }
 
-    // Remaining rounds, loads one round ahead (two register buffers, unrolled by two).
-    for (int r = 1; ok && r * kRing < nst; r += 2) {
-      load_round(wa, r + 1);
-      ok = process_round(wb, r);
-      if (!ok || (r + 1) * kRing >= nst) break;
-      load_round(wb, r + 2);
-      ok = process_round(wa, r + 1);
+    // Remaining stages through the ring, from the words already in registers.
+    bool ok = true;
+#pragma unroll
+    for (int j = kRing; j < kMaxStagesPerCta; ++j) {
+      if (j >= nst || !ok) break;
+      const int slot = j % kRing;
+      uint32_t v[32];
+      expand_stage(w[2 * j], w[2 * j + 1], v);
+      ok = warp_wait(&sh->empty[slot], (uint32_t)((j / kRing) - 1) & 1u, err, abort_flag, lane);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st_x32(lane_base + kRingBase + 32u * slot, v);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->full[slot]);
     }
 
     // Epilogue: this row's 16 partial sums.
     float acc[kTok];
-    {
-      int okw = 1;
-      if (lane == 0) okw = mbar_wait(&sh->dfull, 0, err, abort_flag) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, okw, 0) && ok;
-    }
+    ok = warp_wait(&sh->dfull, 0, err, abort_flag, lane) && ok;
     tc_fence_after();
     {
-      uint32_t d[16];
-      tmem_ld_x16(lane_base, d);
+      // D_2 and D_3 hold data only if the CTA's first stage is a full 64-k stage.
+      const int nacc = ((int64_t)st0 * kStageK + 32 < K) ? kAcc : 2;
+      uint32_t d[kAcc][16];
+#pragma unroll
+      for (int q = 0; q < kAcc; ++q) tmem_ld_x16(lane_base + 16u * q, d[q]);
       tmem_wait_ld();
 #pragma unroll
-      for (int m = 0; m < kTok; ++m) acc[m] = ok ? __uint_as_float(d[m]) : 0.f;
+      for (int m = 0; m < kTok; ++m) {
+        float v = __uint_as_float(d[0][m]) + __uint_as_float(d[1][m]);
+        if (nacc == kAcc) v += __uint_as_float(d[2][m]) + __uint_as_float(d[3][m]);
+        acc[m] = ok ? v : 0.f;
+      }
     }
     if constexpr (!kCluster) {
       if (row_ok) {
-        const float sc = __ldg(g.oscale + n);
 #pragma unroll
         for (int m = 0; m < kTok; ++m) {
           if (m >= mt) break;
           const int64_t off = (m0 + m) * g.ldy + n;
           if (g.y_dtype == OB_OUT_F32)
-            static_cast<float*>(g.Y)[off] = acc[m] * sc;
+            static_cast<float*>(g.Y)[off] = acc[m] * osc;
           else
-            static_cast<__nv_bfloat16*>(g.Y)[off] = __float2bfloat16_rn(acc[m] * sc);
+            static_cast<__nv_bfloat16*>(g.Y)[off] = __float2bfloat16_rn(acc[m] * osc);
         }
       }
     } else {
@@ -277,7 +317,7 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_tc_decode_kernel(SignGemmA
         const int ksub = (k_stage + 32 < K) ? 4 : 2;  // last stage may hold one word
         for (int q = 0; q < ksub; ++q) {
           const uint64_t bdesc = sdesc_kmajor_sw128(xs_atom + 32u * q);
-          mma_bf16_ts(tmem, tmem + 32u + 32u * slot + 8u * q, bdesc, kIdesc, (j > 0 || q > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + 16u * q, tmem + kRingBase + 32u * slot + 8u * q, bdesc, kIdesc, j > 0 ? 1u : 0u);
         }
         mma_commit(&sh->empty[slot]);
       }
@@ -288,19 +328,25 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_tc_decode_kernel(SignGemmA
   }
 
   if constexpr (kCluster) {
-    cluster_sync_all();
     // Rank ks reduces rows [ks*128/ksplit, (ks+1)*128/ksplit) over all CTAs of the cluster.
     const int r0 = kRows * ks / ksplit, r1 = kRows * (ks + 1) / ksplit;
     const int rows = r1 - r0;
+    const int my_r = r0 + tid % rows;  // each thread keeps one row (kThreads is a multiple of rows or more)
+    const float my_osc = (n0 + my_r < g.R) ? __ldg(g.oscale + n0 + my_r) : 0.f;
+    cluster_sync_all();
     if (!*abort_flag) {
       for (int idx = tid; idx < rows * (int)mt; idx += kThreads) {
         const int m = idx / rows;
         const int r = r0 + (idx - m * rows);
         const int64_t n = n0 + r;
         if (n >= g.R) continue;
+        float parts[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) parts[q] = q < ksplit ? ld_dsmem_f32(&sh->part[m][r], (uint32_t)q) : 0.f;
         float s = 0.f;
-        for (int q = 0; q < ksplit; ++q) s += ld_dsmem_f32(&sh->part[m][r], (uint32_t)q);
-        s *= __ldg(g.oscale + n);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) s += parts[q];
+        s *= (r == my_r) ? my_osc : __ldg(g.oscale + n);
         const int64_t off = (m0 + m) * g.ldy + n;
         if (g.y_dtype == OB_OUT_F32)
           static_cast<float*>(g.Y)[off] = s;
@@ -324,14 +370,16 @@ int env_int(const char* name, int dflt) {
   return s ? std::atoi(s) : dflt;
 }
 
-// K-split over the cluster: minimise the per-SM share of the work, prefer fewer splits.
+// K-split over the cluster: with two CTAs per SM, minimise the per-SM share of
+// the work; prefer fewer splits on ties.
 int choose_ksplit(int64_t row_blocks, int stages, int num_sms) {
   const int forced = env_int("OB_DECODE_KSPLIT", 0);
-  int best = 1;
+  auto fits = [&](int ks) { return ks <= stages && (stages + ks - 1) / ks <= kMaxStagesPerCta; };
+  if (forced > 0 && forced <= 8 && fits(forced)) return forced;
+  int best = 0;
   double best_cost = 1e30;
   for (int ks = 1; ks <= 8; ++ks) {
-    if (ks > stages) break;
-    if ((stages + ks - 1) / ks > kMaxStagesPerCta) continue;
+    if (!fits(ks)) continue;
     const int64_t ctas = row_blocks * ks;
     const double cost = (double)((ctas + num_sms - 1) / num_sms) / ks;
     if (cost < best_cost - 1e-9) {
@@ -339,8 +387,6 @@ int choose_ksplit(int64_t row_blocks, int stages, int num_sms) {
       best = ks;
     }
   }
-  if (forced > 0 && forced <= 8 && forced <= stages && (stages + forced - 1) / forced <= kMaxStagesPerCta)
-    best = forced;
   return best;
 }
 
@@ -350,8 +396,8 @@ cudaError_t launch_sign_gemm_tc_decode(const SignGemmArgs& g, const LaunchCtx& c
   const int stages = (int)((g.K + kStageK - 1) / kStageK);
   const int64_t row_blocks = (g.R + kRows - 1) / kRows;
   if (stages == 0 || row_blocks == 0 || g.M == 0) return cudaSuccess;
-  if ((stages + 7) / 8 > kMaxStagesPerCta) return cudaErrorInvalidValue;  // K too large for this kernel
   const int ksplit = choose_ksplit(row_blocks, stages, c.num_sms);
+  if (ksplit == 0) return cudaErrorInvalidValue;  // K too large for one cluster of this kernel
   const size_t smem = 1024 + (size_t)kMaxStagesPerCta * kAtomBytes + sizeof(DecodeShared);
 
   for (int64_t m0 = 0; m0 < g.M; m0 += kTok) {
