@@ -12,6 +12,10 @@
 // Device error word: bits OB_DEVERR_* set by kernels, read and cleared by ob_last_device_error.
 __device__ unsigned g_ob_error_word;
 
+// Static scratch for dbf_linear_noalloc: holds the DBF intermediate for callers
+// that cannot allocate.  Reserved on every device that loads the library.
+static __device__ __align__(256) unsigned char g_dbf_noalloc_scratch[OB_DBF_NOALLOC_SCRATCH_BYTES];
+
 namespace ob {
 namespace {
 
@@ -240,6 +244,33 @@ ob_status dbf_linear(const void* X, int64_t M, int64_t K, const uint32_t* SB_pac
                      void* workspace, size_t ws_bytes, void* stream) {
   return dbf_linear_ex(X, M, K, SB_packed, r, m, SA_packed, N, a, b, Y, y_dtype, workspace, ws_bytes,
                        OB_PATH_AUTO, stream);
+}
+
+ob_status dbf_linear_noalloc(const void* X, int64_t M, int64_t K, const uint32_t* SB_packed, int64_t r,
+                             const float* m, const uint32_t* SA_packed, int64_t N, const float* a, const float* b,
+                             void* Y, int y_dtype, void* stream) {
+  // Size check first, before any CUDA call: the intermediate is M x r bf16.
+  if (M < 0 || r < 0) return OB_ERR_SHAPE;
+  if ((size_t)M * (size_t)r * 2 > (size_t)OB_DBF_NOALLOC_SCRATCH_BYTES) return OB_ERR_WORKSPACE;
+  // Device address of the static scratch on the current device, looked up once per
+  // device with that device current.  The array's name in host code is only a
+  // host-side handle, never a device address.
+  static std::mutex mu;
+  static void* scratch[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return OB_ERR_CUDA;
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!scratch[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_dbf_noalloc_scratch) != cudaSuccess || p == nullptr) return OB_ERR_CUDA;
+      scratch[dev] = p;
+    }
+    ptr = scratch[dev];
+  }
+  return dbf_linear_ex(X, M, K, SB_packed, r, m, SA_packed, N, a, b, Y, y_dtype, ptr,
+                       (size_t)OB_DBF_NOALLOC_SCRATCH_BYTES, OB_PATH_AUTO, stream);
 }
 
 ob_status ob_selftest_timeout(uint64_t limit_ns, void* stream) {

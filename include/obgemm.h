@@ -31,8 +31,10 @@
  *    vectors are fp32, Y is bf16 (round to nearest even) or fp32 by `y_dtype`.
  *  - Pointers are DEVICE pointers unless a parameter says "host".  The caller
  *    owns every buffer; the library allocates no device memory.  It holds
- *    one 4-byte device error word per device (module-scope) and nothing else.
- *    Every device pointer must be 16-byte aligned.
+ *    one 4-byte device error word per device (module-scope) and the static
+ *    scratch array of dbf_linear_noalloc (OB_DBF_NOALLOC_SCRATCH_BYTES per
+ *    device, module-scope), and nothing else.  Every device pointer must be
+ *    16-byte aligned.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Calls are asynchronous and stream-ordered unless noted.
  *  - Errors: argument checks run on the host before any launch and return a
@@ -191,6 +193,38 @@ OB_API ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K,
                         const float* a, const float* b,
                         void* Y, int y_dtype,
                         void* workspace, size_t ws_bytes, int path, void* stream);
+
+/* Size of the static scratch behind dbf_linear_noalloc: M * r * 2 bytes must fit. */
+#define OB_DBF_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/*
+ * dbf_linear for callers that cannot allocate device memory (the pages have no
+ * counterpart; this is a deployment convenience).  Same operation, arguments
+ * and result as dbf_linear, minus the workspace: the M x r intermediate lives
+ * in a static device array of OB_DBF_NOALLOC_SCRATCH_BYTES that the library
+ * reserves on every GPU where it is loaded, for the life of the process.
+ *
+ * Who needs it: code that enqueues work while its stream is being captured
+ * into a CUDA graph (cudaMalloc is not a stream operation, cannot be recorded,
+ * and may synchronise the device, which capture forbids); inference engines
+ * and framework plugins that run against a fixed memory plan and may not
+ * allocate at enqueue time; and callers whose device memory is owned by
+ * another allocator that a raw cudaMalloc would bypass.  This call itself
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  Returns OB_ERR_WORKSPACE, launching nothing, when M * r * 2 bytes
+ * exceed OB_DBF_NOALLOC_SCRATCH_BYTES.  Every call on a device shares the one
+ * array and it keeps the last call's contents (each call overwrites the
+ * intermediate before reading it): calls that may overlap on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller.
+ */
+OB_API ob_status dbf_linear_noalloc(const void* X, int64_t M, int64_t K,
+                                    const uint32_t* SB_packed, int64_t r, const float* m,
+                                    const uint32_t* SA_packed, int64_t N,
+                                    const float* a, const float* b,
+                                    void* Y, int y_dtype, void* stream);
 
 /*
  * Self-test of the bounded-wait machinery (no counterpart on the pages): one
