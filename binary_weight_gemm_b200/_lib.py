@@ -17,7 +17,7 @@ STATUS_NAMES = {
     9: "OB_ERR_UNSUPPORTED", 10: "OB_ERR_DEVICE_BOUNDS",
 }
 OB_OUT_BF16, OB_OUT_F32 = 0, 1
-OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC_DECODE, OB_PATH_TC = 0, 1, 2, 3
+OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC_DECODE, OB_PATH_TC, OB_PATH_MMA_DECODE = 0, 1, 2, 3, 4
 
 # Every function the header declares, with (restype, argtypes).
 _P, _I64, _I, _F, _SZ, _U64 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,

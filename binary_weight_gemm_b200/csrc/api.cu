@@ -90,11 +90,16 @@ ob_status status_of(cudaError_t e) {
 }
 
 ob_status run_sign_gemm(const SignGemmArgs& g, int path, const LaunchCtx& c) {
-  if (path == OB_PATH_AUTO) path = (g.M <= decode_max_m()) ? OB_PATH_TC_DECODE : OB_PATH_TC;
+  // Measured on B200 (4096 x 4096 layer, one call per CUDA-graph node): one token is
+  // fastest on the table-driven CUDA-core kernel, 2..16 tokens on the warp-level
+  // MMA kernel, more on the tcgen05 GEMM.
+  if (path == OB_PATH_AUTO)
+    path = g.M == 1 ? OB_PATH_SIMT : (g.M <= decode_max_m() ? OB_PATH_MMA_DECODE : OB_PATH_TC);
   cudaError_t e;
   switch (path) {
     case OB_PATH_SIMT: e = launch_sign_gemm_simt(g, c); break;
     case OB_PATH_TC_DECODE: e = launch_sign_gemm_tc_decode(g, c); break;
+    case OB_PATH_MMA_DECODE: e = launch_sign_gemm_mma_decode(g, c); break;
     case OB_PATH_TC: e = launch_sign_gemm_tc(g, c); break;
     default: return OB_ERR_UNSUPPORTED;
   }
@@ -184,7 +189,7 @@ ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
                        const float* b, void* Y, int y_dtype, int path, void* stream) {
   if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
-  if (path < OB_PATH_AUTO || path > OB_PATH_TC) return OB_ERR_UNSUPPORTED;
+  if (path < OB_PATH_AUTO || path > OB_PATH_MMA_DECODE) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   if (K > 0 && (!X || !W_packed || !b)) return OB_ERR_NULL;
@@ -213,7 +218,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
                         void* workspace, size_t ws_bytes, int path, void* stream) {
   if (M < 0 || N < 0 || K < 0 || r < 0 || K % 32 != 0 || r % 32 != 0) return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
-  if (path < OB_PATH_AUTO || path > OB_PATH_TC) return OB_ERR_UNSUPPORTED;
+  if (path < OB_PATH_AUTO || path > OB_PATH_MMA_DECODE) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   const bool empty_sum = (K == 0 || r == 0);

@@ -35,6 +35,7 @@ cudaError_t launch_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* ou
 
 cudaError_t launch_sign_gemm_simt(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_tc_decode(const SignGemmArgs& g, const LaunchCtx& c);
+cudaError_t launch_sign_gemm_mma_decode(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c);
 
 // SVID power iteration pieces (see svid.cu).

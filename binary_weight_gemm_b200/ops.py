@@ -15,8 +15,8 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import (OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC,  # noqa: F401
-                   OB_PATH_TC_DECODE, ObError)
+from ._lib import (OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_MMA_DECODE, OB_PATH_SIMT,  # noqa: F401
+                   OB_PATH_TC, OB_PATH_TC_DECODE, ObError)
 
 
 def _stream(stream) -> int:

@@ -82,10 +82,11 @@ typedef enum ob_out_dtype {
 
 /* Kernel choice for ob_linear_ex / dbf_linear_ex. */
 typedef enum ob_path {
-  OB_PATH_AUTO = 0,       /* M <= decode limit: OB_PATH_TC_DECODE, else OB_PATH_TC */
-  OB_PATH_SIMT = 1,       /* CUDA-core select/add mat-vec (any M; slow for M > 4) */
-  OB_PATH_TC_DECODE = 2,  /* tcgen05, signs unpacked into tensor memory, M <= 16 per pass */
-  OB_PATH_TC = 3          /* tcgen05 tiled GEMM for large M (activations by TMA) */
+  OB_PATH_AUTO = 0,        /* M == 1: OB_PATH_SIMT; M <= 16: OB_PATH_MMA_DECODE; else OB_PATH_TC */
+  OB_PATH_SIMT = 1,        /* CUDA-core select/add mat-vec (any M; slow for M > 4) */
+  OB_PATH_TC_DECODE = 2,   /* tcgen05, signs unpacked into tensor memory, M <= 16 per pass */
+  OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA) */
+  OB_PATH_MMA_DECODE = 4   /* warp-level MMA, signs unpacked in registers, M <= 16 per pass */
 } ob_path;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -148,7 +149,8 @@ OB_API ob_status ob_svid_rank1(const float* W, int64_t N, int64_t K,
  *   b         device, fp32 [K] (the page's g).
  *   Y         device, M x N, bf16 or fp32 by y_dtype.
  * K % 32 == 0.  Accumulates in fp32.  Asynchronous.  OB_PATH_AUTO picks the
- * tensor-memory decode kernel for M <= 16 and the tiled tcgen05 GEMM above.
+ * table-driven CUDA-core kernel for M == 1, the warp-level MMA decode kernel for
+ * M <= 16 (OB_DECODE_MAX_M) and the tiled tcgen05 GEMM above.
  */
 OB_API ob_status ob_linear(const void* X, int64_t M, int64_t K,
                     const uint32_t* W_packed, int64_t N,

@@ -9,7 +9,7 @@ from helpers import assert_gemm_close
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc_decode": 2, "tc": 3, "auto": 0}
+PATHS = {"simt": 1, "tc_decode": 2, "tc": 3, "mma_decode": 4, "auto": 0}
 
 
 @pytest.fixture(scope="module")
@@ -39,7 +39,7 @@ def _ref(x, f):
     return oracle.dbf_linear(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"])
 
 
-@pytest.mark.parametrize("path", ["simt", "tc_decode", "tc"])
+@pytest.mark.parametrize("path", ["simt", "tc_decode", "tc", "mma_decode"])
 @pytest.mark.parametrize("M,N,r,K", [(1, 128, 32, 64), (4, 256, 96, 256), (7, 200, 160, 96), (33, 130, 64, 128),
                                      (260, 256, 128, 320)])
 def test_dbf_small_shapes(ops, path, M, N, r, K):

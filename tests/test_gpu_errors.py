@@ -57,6 +57,6 @@ def test_no_device_error_after_normal_work(ops):
     P = ops.ob_pack_signs(W)
     xb, _ = synth.activations(1, 40, 256)
     X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
-    for path in (0, 1, 2, 3):
+    for path in (0, 1, 2, 3, 4):
         ops.ob_linear(X, P, a, b, path=path)
     assert ops.ob_last_device_error() == 0

@@ -15,7 +15,7 @@ from helpers import assert_gemm_close, oracle_svid
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc_decode": 2, "tc": 3}
+PATHS = {"simt": 1, "tc_decode": 2, "tc": 3, "mma_decode": 4}
 
 
 @pytest.fixture(scope="module")
@@ -147,7 +147,7 @@ def test_linear_degenerate_sizes(ops):
 
 # ---------------------------------------------------------------- full-size workloads
 
-@pytest.mark.parametrize("path", ["tc_decode", "simt"])
+@pytest.mark.parametrize("path", ["mma_decode", "tc_decode", "simt"])
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_decode_workload_full(ops, path, M):
     # OneBit decode GEMV: X M x 4096, W 4096 x 4096 -> 2 MiB packed, a, b from SVID.
