@@ -18,8 +18,8 @@
 //    signs cost no shared-memory bandwidth.
 //  * warp 9 (one lane): tcgen05.mma kind::f16, M=128, N=256, K=16, fp32
 //    accumulators in TMEM (256 columns); tcgen05.commit releases ring slots.
-//  * warps 4-7: epilogue, tcgen05.ld of the accumulator, * oscale, bf16/fp32
-//    stores (each warp store covers 32 consecutive outputs of one token row).
+//  * warps 4-7: epilogue, tcgen05.ld of the accumulator, * oscale, transposed
+//    through shared memory into 16-byte stores along Y's rows.
 // Every mbarrier wait is bounded (see ob_device.cuh).
 #include <algorithm>
 #include <cstring>
@@ -39,7 +39,7 @@ constexpr int kBK = 64;        // k per stage
 constexpr int kStages = 4;
 constexpr int kThreads = 320;  // 10 warps
 constexpr uint32_t kXStageBytes = kTok * kBK * 2;  // 32 KB
-constexpr int kTmemCols = 512;                     // D [0,256), A slots 256 + 32*s
+constexpr int kTmemCols = 512;                     // D [0,256), A slots 256 + 32*s (s < 4)
 constexpr uint32_t kIdesc = idesc_bf16_f32(kRows, kTok);
 constexpr int64_t kMaxK = 24576;                   // iscale pairs staged in shared memory
 
@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
   uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   TcShared* sh = reinterpret_cast<TcShared*>(xs + (size_t)kStages * kXStageBytes);
   uint32_t* bpair = reinterpret_cast<uint32_t*>(sh + 1);  // [K/2] bf16x2 (iscale[2i], iscale[2i+1])
+  // Epilogue transpose scratch: 4 warps x 32 x 33 floats, after the scale pairs.
+  float* epi_scratch = reinterpret_cast<float*>(bpair + (((g.K + 1) / 2 + 3) & ~int64_t(3)));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t K = g.K, Wd = K / 32;
@@ -104,83 +106,143 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
 
   if (warp < 4) {
     // ------------------------------------------------ A producer: signs (x) input scale -> TMEM
+    // Sign words are fetched a whole group of four stages (8 words) ahead, so an L2
+    // round trip is always hidden behind four stages of MMAs.
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const bool vec = (Wd & 3) == 0;
     int64_t gstage = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
       const int64_t n = (tile % n_blocks) * kRows + tid;
       const bool row_ok = n < g.R;
       const uint32_t* srow = g.S + (row_ok ? n : 0) * Wd;
-      uint32_t nw0 = row_ok ? __ldg(srow) : 0u;
-      uint32_t nw1 = (row_ok && Wd > 1) ? __ldg(srow + 1) : 0u;
-      for (int kb = 0; kb < nkb; ++kb, ++gstage) {
-        const uint32_t w0 = nw0, w1 = nw1;
-        const int64_t wn = 2 * (int64_t)(kb + 1);  // prefetch the next stage's words
-        nw0 = (row_ok && wn < Wd) ? __ldg(srow + wn) : 0u;
-        nw1 = (row_ok && wn + 1 < Wd) ? __ldg(srow + wn + 1) : 0u;
-        const int s = (int)(gstage % kStages);
-        if (gstage >= kStages) {
-          ok = wait_warp(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag, lane);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        const uint4* bp = reinterpret_cast<const uint4*>(bpair + (int64_t)kb * (kBK / 2));
-        const bool full_stage = (int64_t)(kb + 1) * kBK <= K;
-        uint32_t v[32];
+      auto load_group = [&](int64_t grp, uint32_t (&wv)[8]) {
+        const int64_t w0 = grp * 8;
+        if (vec) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint4 b4 = make_uint4(0, 0, 0, 0);
-          if (full_stage || q < 4) b4 = bp[q];  // a trailing half stage reads 32 k only
-          const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = q * 4 + e;          // column: k = 2c, 2c+1 within the stage
-            const uint32_t w = c < 16 ? w0 : w1;
-            const int i = (2 * c) & 31;       // bit of k = 2c
-            const uint32_t lo = i <= 15 ? (w << (15 - i)) : (w >> (i - 15));
-            const uint32_t hi = w << (30 - i);
-            v[c] = bb[e] ^ (lo & 0x8000u) ^ (hi & 0x80000000u);
+          for (int h = 0; h < 2; ++h) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (row_ok && w0 + 4 * h < Wd) v = __ldg(reinterpret_cast<const uint4*>(srow + w0) + h);
+            wv[4 * h] = v.x; wv[4 * h + 1] = v.y; wv[4 * h + 2] = v.z; wv[4 * h + 3] = v.w;
           }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) wv[i] = (row_ok && w0 + i < Wd) ? __ldg(srow + w0 + i) : 0u;
         }
-        tmem_st_x32(lane_base + 256u + 32u * s, v);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->afull[s]);
+      };
+      uint32_t cur[8], nxt[8];
+      load_group(0, cur);
+      const int ngroups = (nkb + 3) / 4;
+      for (int grp = 0; grp < ngroups && ok; ++grp) {
+        load_group(grp + 1, nxt);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int kb = grp * 4 + i;
+          if (kb >= nkb) break;
+          const uint32_t w0 = cur[2 * i], w1 = cur[2 * i + 1];
+          const int s = (int)(gstage % kStages);
+          if (gstage >= kStages) {
+            ok = wait_warp(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag, lane);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          const uint4* bp = reinterpret_cast<const uint4*>(bpair + (int64_t)kb * (kBK / 2));
+          const bool full_stage = (int64_t)(kb + 1) * kBK <= K;
+          uint32_t v[32];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            uint4 b4 = make_uint4(0, 0, 0, 0);
+            if (full_stage || q < 4) b4 = bp[q];  // a trailing half stage reads 32 k only
+            const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = q * 4 + e;          // column: k = 2c, 2c+1 within the stage
+              const uint32_t w = c < 16 ? w0 : w1;
+              const int ib = (2 * c) & 31;      // bit of k = 2c
+              const uint32_t lo = ib <= 15 ? (w << (15 - ib)) : (w >> (ib - 15));
+              const uint32_t hi = w << (30 - ib);
+              v[c] = bb[e] ^ (lo & 0x8000u) ^ (hi & 0x80000000u);
+            }
+          }
+          tmem_st_x32(lane_base + 256u + 32u * s, v);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh->afull[s]);
+          ++gstage;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
       }
     }
   } else if (warp < 8) {
     // ------------------------------------------------ epilogue
+    // A thread holds one weight row of the accumulator and 32 token columns per
+    // tcgen05.ld.  Each warp transposes its 32 x 32 block through a small shared
+    // scratch so that every store is a 16-byte piece of one Y row (8 bf16 or 4
+    // fp32 consecutive outputs), instead of 32 scattered 2-byte stores.
     const int q = warp - 4;  // TMEM lane quadrant
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    float* scr = epi_scratch + q * (32 * 33);
+    const bool f32 = g.y_dtype == OB_OUT_F32;
+    const bool vec_ok = (g.ldy % (f32 ? 4 : 8)) == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0;
     pdl_wait();
     int64_t it = 0;
     for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
       if (!wait_warp(&sh->dfull, (uint32_t)it & 1u, err, abort_flag, lane)) break;
       tc_fence_after();
       const int64_t m0 = (tile / n_blocks) * kTok;
-      const int64_t n = (tile % n_blocks) * kRows + q * 32 + lane;
-      const bool row_ok = n < g.R;
-      const float sc = row_ok ? __ldg(g.oscale + n) : 0.f;
+      const int64_t nq = (tile % n_blocks) * kRows + q * 32;  // this warp's 32 weight rows
+      const float sc = (nq + lane < g.R) ? __ldg(g.oscale + nq + lane) : 0.f;
 #pragma unroll 1
       for (int c = 0; c < kTok / 32; ++c) {
         uint32_t d[32];
         tmem_ld_x32(lane_base + 32u * c, d);
         tmem_wait_ld();
-        if (row_ok) {
+        // scr[token][row], row = lane (pitch 33 floats: conflict-free both ways)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int64_t m = m0 + 32 * c + i;
+        for (int i = 0; i < 32; ++i) scr[i * 33 + lane] = __uint_as_float(d[i]) * sc;
+        __syncwarp();
+        const int64_t mc = m0 + 32 * c;
+        if (f32) {
+          // 32 tokens x 8 pieces of 4 outputs: lane -> (token, piece)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int v = lane + 32 * i, tok = v >> 3, pc = v & 7;
+            const int64_t m = mc + tok, n = nq + 4 * pc;
             if (m < g.M) {
-              const float y = __uint_as_float(d[i]) * sc;
-              const int64_t off = m * g.ldy + n;
-              if (g.y_dtype == OB_OUT_F32)
-                static_cast<float*>(g.Y)[off] = y;
-              else
-                static_cast<__nv_bfloat16*>(g.Y)[off] = __float2bfloat16_rn(y);
+              const float* src = scr + tok * 33 + 4 * pc;
+              float* dst = static_cast<float*>(g.Y) + m * g.ldy + n;
+              if (vec_ok && n + 4 <= g.R) {
+                *reinterpret_cast<float4*>(dst) = make_float4(src[0], src[1], src[2], src[3]);
+              } else {
+                for (int e = 0; e < 4; ++e)
+                  if (n + e < g.R) dst[e] = src[e];
+              }
+            }
+          }
+        } else {
+          // 32 tokens x 4 pieces of 8 outputs
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int v = lane + 32 * i, tok = v >> 2, pc = v & 3;
+            const int64_t m = mc + tok, n = nq + 8 * pc;
+            if (m < g.M) {
+              const float* src = scr + tok * 33 + 8 * pc;
+              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.Y) + m * g.ldy + n;
+              if (vec_ok && n + 8 <= g.R) {
+                uint4 o;
+                o.x = pack_bf16x2(src[0], src[1]); o.y = pack_bf16x2(src[2], src[3]);
+                o.z = pack_bf16x2(src[4], src[5]); o.w = pack_bf16x2(src[6], src[7]);
+                *reinterpret_cast<uint4*>(dst) = o;
+              } else {
+                for (int e = 0; e < 8; ++e)
+                  if (n + e < g.R) dst[e] = __float2bfloat16_rn(src[e]);
+              }
             }
           }
         }
+        __syncwarp();  // scr is rewritten by the next chunk
       }
       tc_fence_before();
       __syncwarp();
@@ -224,11 +286,20 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
           ok = mbar_wait(&sh->xfull[s], par, err, abort_flag) && mbar_wait(&sh->afull[s], par, err, abort_flag);
           if (!ok) break;
           tc_fence_after();
+          // All four descriptors are formed before the first MMA of the stage, each in
+          // its own register, and the MMAs are unrolled: an MMA reads its operand
+          // registers after issue, so rewriting them for the next MMA would stall.
           const uint32_t xa = smem_u32(xs) + (uint32_t)s * kXStageBytes;
-          const int ksub = ((int64_t)(kb + 1) * kBK <= K) ? 4 : 2;
-          for (int q = 0; q < ksub; ++q)
-            mma_bf16_ts(tmem, tmem + 256u + 32u * s + 8u * q, sdesc_kmajor_sw128(xa + 32u * q), kIdesc,
-                        (kb > 0 || q > 0) ? 1u : 0u);
+          const uint32_t aa = tmem + 256u + 32u * (uint32_t)s;
+          const uint64_t b0 = sdesc_kmajor_sw128(xa), b1 = sdesc_kmajor_sw128(xa + 32u);
+          const uint64_t b2 = sdesc_kmajor_sw128(xa + 64u), b3 = sdesc_kmajor_sw128(xa + 96u);
+          const uint32_t acc0 = kb > 0 ? 1u : 0u;
+          mma_bf16_ts(tmem, aa, b0, kIdesc, acc0);
+          mma_bf16_ts(tmem, aa + 8u, b1, kIdesc, 1u);
+          if ((int64_t)(kb + 1) * kBK <= K) {  // a trailing half stage holds 32 k
+            mma_bf16_ts(tmem, aa + 16u, b2, kIdesc, 1u);
+            mma_bf16_ts(tmem, aa + 24u, b3, kIdesc, 1u);
+          }
           mma_commit(&sh->empty[s]);
         }
         mma_commit(&sh->dfull);
@@ -285,7 +356,8 @@ cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
 
   const int64_t tiles = ((g.M + kTok - 1) / kTok) * ((g.R + kRows - 1) / kRows);
   const int grid = (int)std::min<int64_t>(tiles, c.num_sms);
-  const size_t smem = 1024 + (size_t)kStages * kXStageBytes + sizeof(TcShared) + sizeof(uint32_t) * ((g.K + 1) / 2);
+  const size_t smem = 1024 + (size_t)kStages * kXStageBytes + sizeof(TcShared) +
+                      sizeof(uint32_t) * ((((g.K + 1) / 2) + 3) & ~int64_t(3)) + sizeof(float) * 4 * 32 * 33;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
