@@ -9,16 +9,17 @@
 //
 // Persistent, warp-specialised kernel, one CTA per SM, output tile 128 weight
 // rows x 256 tokens:
-//  * warp 8 (one lane): TMA loads of the activation tile (256 tokens x 64 k,
+//  * warp 12 (one lane): TMA loads of the activation tile (256 tokens x 64 k,
 //    bf16, 128-byte swizzle) into a 4-deep shared-memory ring.  This is the MMA's
 //    B operand; the activations are never touched by a thread.
 //  * warps 0-3: one thread per weight row expands two packed words (64 k) into
 //    32 TMEM columns of bf16 pairs (+/-bf16(b_k), +/-bf16(b_k+1)) with
 //    tcgen05.st.  This is the MMA's A operand in tensor memory, so the expanded
 //    signs cost no shared-memory bandwidth.
-//  * warp 9 (one lane): tcgen05.mma kind::f16, M=128, N=256, K=16, fp32
+//  * warp 13 (one lane): tcgen05.mma kind::f16, M=128, N=256, K=16, fp32
 //    accumulators in TMEM (256 columns); tcgen05.commit releases ring slots.
-//  * warps 4-7: epilogue, tcgen05.ld of the accumulator, * oscale, transposed
+//  * warps 4-11: epilogue, two warps per TMEM lane quadrant (each drains half of
+//    the token columns): tcgen05.ld of the accumulator, * oscale, transposed
 //    through shared memory into 16-byte stores along Y's rows.
 // Every mbarrier wait is bounded (see ob_device.cuh).
 #include <algorithm>
@@ -37,7 +38,7 @@ constexpr int kRows = 128;     // MMA M (weight rows)
 constexpr int kTok = 256;      // MMA N (tokens)
 constexpr int kBK = 64;        // k per stage
 constexpr int kStages = 4;
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 448;  // 14 warps
 constexpr uint32_t kXStageBytes = kTok * kBK * 2;  // 32 KB
 constexpr int kTmemCols = 512;                     // D [0,256), A slots 256 + 32*s (s < 4)
 constexpr uint32_t kIdesc = idesc_bf16_f32(kRows, kTok);
@@ -66,7 +67,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
   uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   TcShared* sh = reinterpret_cast<TcShared*>(xs + (size_t)kStages * kXStageBytes);
   uint32_t* bpair = reinterpret_cast<uint32_t*>(sh + 1);  // [K/2] bf16x2 (iscale[2i], iscale[2i+1])
-  // Epilogue transpose scratch: 4 warps x 32 x 33 floats, after the scale pairs.
+  // Epilogue transpose scratch: 8 warps x 32 x 33 floats, after the scale pairs.
   float* epi_scratch = reinterpret_cast<float*>(bpair + (((g.K + 1) / 2 + 3) & ~int64_t(3)));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
       mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->dfull, 1);
-    mbar_init(&sh->dempty, 4);
+    mbar_init(&sh->dempty, 8);
     sh->abort_flag = 0;
     fence_mbar_init();
   }
@@ -93,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     const float hi = g.iscale ? __ldg(g.iscale + 2 * i + 1) : 1.f;
     bpair[i] = pack_bf16x2(lo, hi);
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(&sh->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -175,15 +176,16 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
         for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------ epilogue
     // A thread holds one weight row of the accumulator and 32 token columns per
     // tcgen05.ld.  Each warp transposes its 32 x 32 block through a small shared
     // scratch so that every store is a 16-byte piece of one Y row (8 bf16 or 4
     // fp32 consecutive outputs), instead of 32 scattered 2-byte stores.
-    const int q = warp - 4;  // TMEM lane quadrant
+    const int q = warp & 3;               // TMEM lane quadrant
+    const int half = (warp - 4) >> 2;     // which half of the token columns
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    float* scr = epi_scratch + q * (32 * 33);
+    float* scr = epi_scratch + (warp - 4) * (32 * 33);
     const bool f32 = g.y_dtype == OB_OUT_F32;
     const bool vec_ok = (g.ldy % (f32 ? 4 : 8)) == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0;
     pdl_wait();
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
       const int64_t nq = (tile % n_blocks) * kRows + q * 32;  // this warp's 32 weight rows
       const float sc = (nq + lane < g.R) ? __ldg(g.oscale + nq + lane) : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < kTok / 32; ++c) {
+      for (int c = half * (kTok / 64); c < (half + 1) * (kTok / 64); ++c) {
         uint32_t d[32];
         tmem_ld_x32(lane_base + 32u * c, d);
         tmem_wait_ld();
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->dempty);
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -357,7 +359,7 @@ cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
   const int64_t tiles = ((g.M + kTok - 1) / kTok) * ((g.R + kRows - 1) / kRows);
   const int grid = (int)std::min<int64_t>(tiles, c.num_sms);
   const size_t smem = 1024 + (size_t)kStages * kXStageBytes + sizeof(TcShared) +
-                      sizeof(uint32_t) * ((((g.K + 1) / 2) + 3) & ~int64_t(3)) + sizeof(float) * 4 * 32 * 33;
+                      sizeof(uint32_t) * ((((g.K + 1) / 2) + 3) & ~int64_t(3)) + sizeof(float) * 8 * 32 * 33;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
