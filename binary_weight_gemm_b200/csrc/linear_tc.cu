@@ -45,8 +45,7 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(kRows, kTok);
 constexpr int64_t kMaxK = 24576;                   // iscale pairs staged in shared memory
 
 struct __align__(128) TcShared {  // 128-byte size keeps the bf16x2 table after it 16-byte aligned
-  uint64_t xfull[kStages];
-  uint64_t afull[kStages];
+  uint64_t full[kStages];   // X tile landed (TMA transaction bytes) and all four A warps stored
   uint64_t empty[kStages];
   uint64_t dfull;
   uint64_t dempty;
@@ -79,8 +78,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sh->xfull[s], 1);
-      mbar_init(&sh->afull[s], 4);
+      mbar_init(&sh->full[s], 5);  // the TMA thread's expect-tx arrival + one per A warp
       mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->dfull, 1);
@@ -169,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->afull[s]);
+          if (lane == 0) mbar_arrive(&sh->full[s]);
           ++gstage;
         }
 #pragma unroll
@@ -265,8 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
             ok = mbar_wait(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag);
             if (!ok) break;
           }
-          mbar_arrive_expect_tx(&sh->xfull[s], kXStageBytes);
-          tma_load_2d(xs + (size_t)s * kXStageBytes, &tmap_x, &sh->xfull[s], kb * kBK, m0);
+          mbar_arrive_expect_tx(&sh->full[s], kXStageBytes);
+          tma_load_2d(xs + (size_t)s * kXStageBytes, &tmap_x, &sh->full[s], kb * kBK, m0);
         }
       }
     }
@@ -285,7 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
         for (int kb = 0; kb < nkb; ++kb, ++gstage) {
           const int s = (int)(gstage % kStages);
           const uint32_t par = (uint32_t)(gstage / kStages) & 1u;
-          ok = mbar_wait(&sh->xfull[s], par, err, abort_flag) && mbar_wait(&sh->afull[s], par, err, abort_flag);
+          // One barrier per stage for both operands: a second wait costs the issuing
+          // thread about a hundred cycles per stage.
+          ok = mbar_wait(&sh->full[s], par, err, abort_flag);
           if (!ok) break;
           tc_fence_after();
           // All four descriptors are formed before the first MMA of the stage, each in
