@@ -37,21 +37,39 @@ namespace {
 constexpr int kRows = 128;     // MMA M (weight rows)
 constexpr int kTok = 256;      // MMA N (tokens)
 constexpr int kBK = 64;        // k per stage
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;
 constexpr int kThreads = 448;  // 14 warps
-constexpr uint32_t kXStageBytes = kTok * kBK * 2;  // 32 KB
-constexpr int kTmemCols = 512;                     // D [0,256), A slots 256 + 32*s (s < 4)
+constexpr uint32_t kXStageBytes = kTok * kBK * 2;   // 32 KB
+constexpr uint32_t kOutTileBytes = kTok * kRows * 2;  // 64 KB: bf16 output tile staged for the TMA store
+constexpr int kTmemCols = 512;                      // D [0,256), A slots 256 + 32*s (s < 4)
 constexpr uint32_t kIdesc = idesc_bf16_f32(kRows, kTok);
-constexpr int64_t kMaxK = 24576;                   // iscale pairs staged in shared memory
+// iscale pairs live in shared memory (2 bytes per k): four ring stages fit up to
+// K = 16384, three up to K = 32768.
+constexpr int64_t kMaxK4 = 16384;
+constexpr int64_t kMaxK = 32768;
 
 struct __align__(128) TcShared {  // 128-byte size keeps the bf16x2 table after it 16-byte aligned
-  uint64_t full[kStages];   // X tile landed (TMA transaction bytes) and all four A warps stored
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];   // X tile landed (TMA transaction bytes) and all four A warps stored
+  uint64_t empty[kMaxStages];
   uint64_t dfull;
   uint64_t dempty;
+  uint64_t stg_full;           // all eight epilogue warps wrote their part of the output tile
+  uint64_t stg_free;           // the TMA store has read the output tile
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// Separates the even and odd bits of a word: bit j of the result's low half is
+// bit 2j of w, bit 16+j is bit 2j+1.  Four exchanges of bit groups (1, 2, 4 and
+// 8 bits wide) between neighbouring positions.
+__host__ __device__ __forceinline__ uint32_t unzip_bits(uint32_t w) {
+  uint32_t t;
+  t = (w ^ (w >> 1)) & 0x22222222u; w ^= t ^ (t << 1);
+  t = (w ^ (w >> 2)) & 0x0C0C0C0Cu; w ^= t ^ (t << 2);
+  t = (w ^ (w >> 4)) & 0x00F000F0u; w ^= t ^ (t << 4);
+  t = (w ^ (w >> 8)) & 0x0000FF00u; w ^= t ^ (t << 8);
+  return w;
+}
 
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, unsigned* err, volatile int* abort_flag,
                                           int lane) {
@@ -60,14 +78,16 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, unsign
   return __shfl_sync(0xffffffffu, okw, 0) != 0;
 }
 
+template <int kStages>
 __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                                                                    SignGemmArgs g, unsigned* err) {
+                                                                    const __grid_constant__ CUtensorMap tmap_y,
+                                                                    SignGemmArgs g, int tma_store, unsigned* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // [ring: kStages x 32 KB][output tile 64 KB][TcShared][iscale pairs]
   uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  TcShared* sh = reinterpret_cast<TcShared*>(xs + (size_t)kStages * kXStageBytes);
+  uint8_t* out_tile = xs + (size_t)kStages * kXStageBytes;
+  TcShared* sh = reinterpret_cast<TcShared*>(out_tile + kOutTileBytes);
   uint32_t* bpair = reinterpret_cast<uint32_t*>(sh + 1);  // [K/2] bf16x2 (iscale[2i], iscale[2i+1])
-  // Epilogue transpose scratch: 8 warps x 32 x 33 floats, after the scale pairs.
-  float* epi_scratch = reinterpret_cast<float*>(bpair + (((g.K + 1) / 2 + 3) & ~int64_t(3)));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t K = g.K, Wd = K / 32;
@@ -83,6 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     }
     mbar_init(&sh->dfull, 1);
     mbar_init(&sh->dempty, 8);
+    mbar_init(&sh->stg_full, 8);
+    mbar_init(&sh->stg_free, 1);
     sh->abort_flag = 0;
     fence_mbar_init();
   }
@@ -147,6 +169,10 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
           }
           const uint4* bp = reinterpret_cast<const uint4*>(bpair + (int64_t)kb * (kBK / 2));
           const bool full_stage = (int64_t)(kb + 1) * kBK <= K;
+          // Column c of the stage holds k = 2c, 2c+1.  After unzip_bits, bit j of a
+          // word's low half is its bit 2j and bit 16+j its bit 2j+1, so one shift
+          // puts both signs of a pair on the bf16 sign bits 15 and 31.
+          const uint32_t u0 = unzip_bits(w0), u1 = unzip_bits(w1);
           uint32_t v[32];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -155,12 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
             const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int c = q * 4 + e;          // column: k = 2c, 2c+1 within the stage
-              const uint32_t w = c < 16 ? w0 : w1;
-              const int ib = (2 * c) & 31;      // bit of k = 2c
-              const uint32_t lo = ib <= 15 ? (w << (15 - ib)) : (w >> (ib - 15));
-              const uint32_t hi = w << (30 - ib);
-              v[c] = bb[e] ^ (lo & 0x8000u) ^ (hi & 0x80000000u);
+              const int c = q * 4 + e;
+              const uint32_t u = c < 16 ? u0 : u1;
+              v[c] = ((u << (15 - (c & 15))) & 0x80008000u) ^ bb[e];
             }
           }
           tmem_st_x32(lane_base + 256u + 32u * s, v);
@@ -176,77 +199,123 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     }
   } else if (warp < 12) {
     // ------------------------------------------------ epilogue
-    // A thread holds one weight row of the accumulator and 32 token columns per
-    // tcgen05.ld.  Each warp transposes its 32 x 32 block through a small shared
-    // scratch so that every store is a 16-byte piece of one Y row (8 bf16 or 4
-    // fp32 consecutive outputs), instead of 32 scattered 2-byte stores.
+    // Two warps per TMEM lane quadrant; a thread holds one weight row of the
+    // accumulator and reads 32 token columns per tcgen05.ld.
     const int q = warp & 3;               // TMEM lane quadrant
     const int half = (warp - 4) >> 2;     // which half of the token columns
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    float* scr = epi_scratch + (warp - 4) * (32 * 33);
-    const bool f32 = g.y_dtype == OB_OUT_F32;
-    const bool vec_ok = (g.ldy % (f32 ? 4 : 8)) == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0;
+    const int c0 = half * (kTok / 64), c1 = c0 + kTok / 64;
     pdl_wait();
     int64_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
-      if (!wait_warp(&sh->dfull, (uint32_t)it & 1u, err, abort_flag, lane)) break;
-      tc_fence_after();
-      const int64_t m0 = (tile / n_blocks) * kTok;
-      const int64_t nq = (tile % n_blocks) * kRows + q * 32;  // this warp's 32 weight rows
-      const float sc = (nq + lane < g.R) ? __ldg(g.oscale + nq + lane) : 0.f;
+    if (tma_store) {
+      // bf16 Y: the tile is staged in shared memory as [token][row], Y's own
+      // layout, and written by one TMA store that clips the ragged edges.  The
+      // accumulator is released right after its last tcgen05.ld, so the next
+      // tile's MMAs overlap the conversion and the store.
+      uint16_t* col = reinterpret_cast<uint16_t*>(out_tile) + q * 32 + lane;
+      for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+        if (!wait_warp(&sh->dfull, (uint32_t)it & 1u, err, abort_flag, lane)) break;
+        tc_fence_after();
+        if (it > 0 && !wait_warp(&sh->stg_free, (uint32_t)(it - 1) & 1u, err, abort_flag, lane)) break;
+        const int64_t m0 = (tile / n_blocks) * kTok;
+        const int64_t n0 = (tile % n_blocks) * kRows;
+        const int64_t nr = n0 + q * 32 + lane;
+        const float sc = nr < g.R ? __ldg(g.oscale + nr) : 0.f;
 #pragma unroll 1
-      for (int c = half * (kTok / 64); c < (half + 1) * (kTok / 64); ++c) {
-        uint32_t d[32];
-        tmem_ld_x32(lane_base + 32u * c, d);
-        tmem_wait_ld();
-        // scr[token][row], row = lane (pitch 33 floats: conflict-free both ways)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) scr[i * 33 + lane] = __uint_as_float(d[i]) * sc;
-        __syncwarp();
-        const int64_t mc = m0 + 32 * c;
-        if (f32) {
-          // 32 tokens x 8 pieces of 4 outputs: lane -> (token, piece)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int v = lane + 32 * i, tok = v >> 3, pc = v & 7;
-            const int64_t m = mc + tok, n = nq + 4 * pc;
-            if (m < g.M) {
-              const float* src = scr + tok * 33 + 4 * pc;
-              float* dst = static_cast<float*>(g.Y) + m * g.ldy + n;
-              if (vec_ok && n + 4 <= g.R) {
-                *reinterpret_cast<float4*>(dst) = make_float4(src[0], src[1], src[2], src[3]);
-              } else {
-                for (int e = 0; e < 4; ++e)
-                  if (n + e < g.R) dst[e] = src[e];
-              }
-            }
+        for (int c = c0; c < c1; ++c) {
+          uint32_t d[32];
+          tmem_ld_x32(lane_base + 32u * c, d);
+          tmem_wait_ld();
+          if (c == c1 - 1) {  // this warp's last read of the accumulator
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh->dempty);
           }
-        } else {
-          // 32 tokens x 4 pieces of 8 outputs
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int v = lane + 32 * i, tok = v >> 2, pc = v & 3;
-            const int64_t m = mc + tok, n = nq + 8 * pc;
-            if (m < g.M) {
-              const float* src = scr + tok * 33 + 8 * pc;
-              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.Y) + m * g.ldy + n;
-              if (vec_ok && n + 8 <= g.R) {
-                uint4 o;
-                o.x = pack_bf16x2(src[0], src[1]); o.y = pack_bf16x2(src[2], src[3]);
-                o.z = pack_bf16x2(src[4], src[5]); o.w = pack_bf16x2(src[6], src[7]);
-                *reinterpret_cast<uint4*>(dst) = o;
-              } else {
-                for (int e = 0; e < 8; ++e)
-                  if (n + e < g.R) dst[e] = __float2bfloat16_rn(src[e]);
-              }
-            }
-          }
+          for (int i = 0; i < 32; ++i)
+            col[(32 * c + i) * kRows] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(d[i]) * sc));
         }
-        __syncwarp();  // scr is rewritten by the next chunk
+        fence_proxy_async_smem();  // the tile is read by the TMA (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->stg_full);
+        if (warp == 4 && lane == 0) {
+          if (mbar_wait(&sh->stg_full, (uint32_t)it & 1u, err, abort_flag)) {
+            tma_store_2d(&tmap_y, out_tile, (int32_t)n0, (int32_t)m0);
+            bulk_commit_group();
+            bulk_wait_read_all();
+          }
+          mbar_arrive(&sh->stg_free);
+        }
+        __syncwarp();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->dempty);
+      if (warp == 4 && lane == 0) bulk_wait_all();
+    } else {
+      // fp32 Y, or a Y the TMA cannot address: each warp transposes its 32 x 32
+      // blocks through shared memory so that every store is a 16-byte piece of
+      // one Y row (8 bf16 or 4 fp32 consecutive outputs).
+      float* scr = reinterpret_cast<float*>(out_tile) + (warp - 4) * (32 * 33);
+      const bool f32 = g.y_dtype == OB_OUT_F32;
+      const bool vec_ok = (g.ldy % (f32 ? 4 : 8)) == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0;
+      for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+        if (!wait_warp(&sh->dfull, (uint32_t)it & 1u, err, abort_flag, lane)) break;
+        tc_fence_after();
+        const int64_t m0 = (tile / n_blocks) * kTok;
+        const int64_t nq = (tile % n_blocks) * kRows + q * 32;  // this warp's 32 weight rows
+        const float sc = (nq + lane < g.R) ? __ldg(g.oscale + nq + lane) : 0.f;
+#pragma unroll 1
+        for (int c = c0; c < c1; ++c) {
+          uint32_t d[32];
+          tmem_ld_x32(lane_base + 32u * c, d);
+          tmem_wait_ld();
+          // scr[token][row], row = lane (pitch 33 floats: conflict-free both ways)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) scr[i * 33 + lane] = __uint_as_float(d[i]) * sc;
+          __syncwarp();
+          const int64_t mc = m0 + 32 * c;
+          if (f32) {
+            // 32 tokens x 8 pieces of 4 outputs: lane -> (token, piece)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int v = lane + 32 * i, tok = v >> 3, pc = v & 7;
+              const int64_t m = mc + tok, n = nq + 4 * pc;
+              if (m < g.M) {
+                const float* src = scr + tok * 33 + 4 * pc;
+                float* dst = static_cast<float*>(g.Y) + m * g.ldy + n;
+                if (vec_ok && n + 4 <= g.R) {
+                  *reinterpret_cast<float4*>(dst) = make_float4(src[0], src[1], src[2], src[3]);
+                } else {
+                  for (int e = 0; e < 4; ++e)
+                    if (n + e < g.R) dst[e] = src[e];
+                }
+              }
+            }
+          } else {
+            // 32 tokens x 4 pieces of 8 outputs
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int v = lane + 32 * i, tok = v >> 2, pc = v & 3;
+              const int64_t m = mc + tok, n = nq + 8 * pc;
+              if (m < g.M) {
+                const float* src = scr + tok * 33 + 8 * pc;
+                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.Y) + m * g.ldy + n;
+                if (vec_ok && n + 8 <= g.R) {
+                  uint4 o;
+                  o.x = pack_bf16x2(src[0], src[1]); o.y = pack_bf16x2(src[2], src[3]);
+                  o.z = pack_bf16x2(src[4], src[5]); o.w = pack_bf16x2(src[6], src[7]);
+                  *reinterpret_cast<uint4*>(dst) = o;
+                } else {
+                  for (int e = 0; e < 8; ++e)
+                    if (n + e < g.R) dst[e] = __float2bfloat16_rn(src[e]);
+                }
+              }
+            }
+          }
+          __syncwarp();  // scr is rewritten by the next chunk
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->dempty);
+      }
     }
   } else if (warp == 12) {
     // ------------------------------------------------ TMA producer
@@ -272,7 +341,13 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
   } else {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int64_t gstage = 0, it = 0;
+      // Descriptors of ring slot 0; slot s adds s * kXStageBytes to the start
+      // address field (address >> 4, no carry out of its 14 bits below 256 KB).
+      const uint32_t xa0 = smem_u32(xs);
+      const uint64_t d0 = sdesc_kmajor_sw128(xa0), d1 = sdesc_kmajor_sw128(xa0 + 32u);
+      const uint64_t d2 = sdesc_kmajor_sw128(xa0 + 64u), d3 = sdesc_kmajor_sw128(xa0 + 96u);
+      uint32_t s = 0, phase = 0;
+      int64_t it = 0;
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++it) {
         if (it > 0) {
@@ -280,29 +355,29 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
           if (!ok) break;
           tc_fence_after();
         }
-        for (int kb = 0; kb < nkb; ++kb, ++gstage) {
-          const int s = (int)(gstage % kStages);
-          const uint32_t par = (uint32_t)(gstage / kStages) & 1u;
+        for (int kb = 0; kb < nkb; ++kb) {
           // One barrier per stage for both operands: a second wait costs the issuing
           // thread about a hundred cycles per stage.
-          ok = mbar_wait(&sh->full[s], par, err, abort_flag);
+          ok = mbar_wait(&sh->full[s], phase, err, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          // All four descriptors are formed before the first MMA of the stage, each in
+          // The four descriptors are ready before the first MMA of the stage, each in
           // its own register, and the MMAs are unrolled: an MMA reads its operand
           // registers after issue, so rewriting them for the next MMA would stall.
-          const uint32_t xa = smem_u32(xs) + (uint32_t)s * kXStageBytes;
-          const uint32_t aa = tmem + 256u + 32u * (uint32_t)s;
-          const uint64_t b0 = sdesc_kmajor_sw128(xa), b1 = sdesc_kmajor_sw128(xa + 32u);
-          const uint64_t b2 = sdesc_kmajor_sw128(xa + 64u), b3 = sdesc_kmajor_sw128(xa + 96u);
-          const uint32_t acc0 = kb > 0 ? 1u : 0u;
-          mma_bf16_ts(tmem, aa, b0, kIdesc, acc0);
+          const uint64_t so = (uint64_t)(s * (kXStageBytes >> 4));
+          const uint64_t b0 = d0 + so, b1 = d1 + so, b2 = d2 + so, b3 = d3 + so;
+          const uint32_t aa = tmem + 256u + 32u * s;
+          mma_bf16_ts(tmem, aa, b0, kIdesc, kb > 0 ? 1u : 0u);
           mma_bf16_ts(tmem, aa + 8u, b1, kIdesc, 1u);
           if ((int64_t)(kb + 1) * kBK <= K) {  // a trailing half stage holds 32 k
             mma_bf16_ts(tmem, aa + 16u, b2, kIdesc, 1u);
             mma_bf16_ts(tmem, aa + 24u, b3, kIdesc, 1u);
           }
           mma_commit(&sh->empty[s]);
+          if (++s == (uint32_t)kStages) {
+            s = 0;
+            phase ^= 1u;
+          }
         }
         mma_commit(&sh->dfull);
       }
@@ -345,21 +420,37 @@ cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
   EncodeTiledFn encode = get_encode_fn();
   if (!encode) return cudaErrorNotSupported;
 
-  CUtensorMap tmap;
-  std::memset(&tmap, 0, sizeof(tmap));
-  const cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.M};
-  const cuuint64_t strides[1] = {(cuuint64_t)g.K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kTok};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(g.X), dims, strides, box,
-                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  CUtensorMap tmap_x, tmap_y;
+  std::memset(&tmap_x, 0, sizeof(tmap_x));
+  std::memset(&tmap_y, 0, sizeof(tmap_y));
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.M};
+    const cuuint64_t strides[1] = {(cuuint64_t)g.K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kTok};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(g.X), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  // bf16 Y whose rows start on 16-byte boundaries is written by TMA stores.
+  int tma_store = 0;
+  if (g.y_dtype == OB_OUT_BF16 && g.ldy % 8 == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0) {
+    const cuuint64_t dims[2] = {(cuuint64_t)g.R, (cuuint64_t)g.M};
+    const cuuint64_t strides[1] = {(cuuint64_t)g.ldy * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kRows, (cuuint32_t)kTok};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&tmap_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.Y, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    tma_store = r == CUDA_SUCCESS ? 1 : 0;
+  }
 
   const int64_t tiles = ((g.M + kTok - 1) / kTok) * ((g.R + kRows - 1) / kRows);
   const int grid = (int)std::min<int64_t>(tiles, c.num_sms);
-  const size_t smem = 1024 + (size_t)kStages * kXStageBytes + sizeof(TcShared) +
-                      sizeof(uint32_t) * ((((g.K + 1) / 2) + 3) & ~int64_t(3)) + sizeof(float) * 8 * 32 * 33;
+  const int stages = g.K <= kMaxK4 ? 4 : 3;
+  const size_t smem = 1024 + (size_t)stages * kXStageBytes + kOutTileBytes + sizeof(TcShared) +
+                      sizeof(uint32_t) * ((((g.K + 1) / 2) + 3) & ~int64_t(3));
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
@@ -375,9 +466,10 @@ cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e = cudaFuncSetAttribute(sign_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = stages == 4 ? sign_gemm_tc_kernel<4> : sign_gemm_tc_kernel<3>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = cudaLaunchKernelEx(&cfg, sign_gemm_tc_kernel, tmap, g, c.err);
+  e = cudaLaunchKernelEx(&cfg, kern, tmap_x, tmap_y, g, tma_store, c.err);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
