@@ -5,8 +5,9 @@ Workload (default): OneBit decode GEMV -- X M x 4096 bf16 ~N(0,1) for M in
 SVID.  One step = one decode token through a pool of L distinct 4096 x 4096
 OneBit layers at each batch size (for M in {1,4,16}: for each layer: ob_linear),
 so every call reads its weights from HBM: the pool (L x 2.1 MB) is larger than
-three times the L2 cache.  The step is captured once as a CUDA graph and
-replayed; inputs are resident in HBM when the timed region starts.
+three times the L2 cache.  Each batch size's pass is captured once as a CUDA
+graph (a decode step runs all layers at one M) and the three are replayed per
+step; inputs are resident in HBM when the timed region starts.
 
   value     HBM GB/s of the step: algorithmic bytes (packed signs + a + b + X + Y
             per call) / device time, summed over ranks, time = max over ranks.
@@ -281,17 +282,27 @@ def run_ours(args, world, rank, local):
             for (P, a, b) in pool:
                 ops.ob_linear(xs[m], P, a, b, out=ys[m], stream=s)
 
-    # Capture one step as a CUDA graph (calls are stream-ordered; no allocation inside).
+    # One CUDA graph per M (calls are stream-ordered; no allocation inside): a decode
+    # step applies every layer at one batch size, and graphs that mix the kernels of
+    # different M lose the programmatic-launch overlap (their shared-memory footprints
+    # differ), which no real decode step would see.  A step replays the three graphs.
+    graphs = {}
     with torch.cuda.stream(stream):
         step(stream)  # warm: first calls set kernel attributes
         stream.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            step(stream)
+        for m in DECODE_MS:
+            graphs[m] = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graphs[m], stream=stream):
+                step(stream, ms=(m,))
     launches_per_step = L * len(DECODE_MS)
 
-    for _ in range(args.warmup):
-        graph.replay()
+    def replay_step():
+        for m in DECODE_MS:
+            graphs[m].replay()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            replay_step()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -300,7 +311,7 @@ def run_ours(args, world, rank, local):
         start.record(stream)
         with torch.cuda.stream(stream):
             for _ in range(args.steps):
-                graph.replay()
+                replay_step()
         end.record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -313,9 +324,7 @@ def run_ours(args, world, rank, local):
     per_m = {}
     for m in DECODE_MS:
         with torch.cuda.stream(stream):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(stream, ms=(m,))
+            g = graphs[m]
             g.replay()
             stream.synchronize()
             reps = max(3, args.steps // 4)
@@ -330,7 +339,6 @@ def run_ours(args, world, rank, local):
                          "weight_gbs": (N_DIM * K_DIM // 8 + 4 * (N_DIM + K_DIM)) / t_call / 1e9,
                          "tflops_equiv": 2 * m * N_DIM * K_DIM / t_call / 1e12,
                          "frac_hbm": decode_call_bytes(m) / t_call / 1e9 / peaks["hbm_gbs"]}
-        del g
 
     # The warp-level MMA kernel forced at M = 1, for comparison with the table-driven kernel AUTO picks.
     with torch.cuda.stream(stream):
@@ -409,7 +417,7 @@ def run_ours(args, world, rank, local):
                        "K": K_DIM, "layers_per_step": L,
                        "l2": f"inputs larger than L2: rotating pool of {L} weight sets "
                              f"({L * decode_call_bytes(0) / 1e6:.0f} MB) per pass",
-                       "graph": "one CUDA graph per step, programmatic dependent launch between calls",
+                       "graph": "one CUDA graph per M (192 calls each), replayed M=1,4,16 per step; programmatic dependent launch between calls",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "tflops_equiv": tflops,
             "per_m": per_m,
@@ -424,7 +432,7 @@ def run_ours(args, world, rank, local):
             "extra": extra,
         }
         print(json.dumps(line), flush=True)
-    del graph
+    graphs.clear()
 
 
 

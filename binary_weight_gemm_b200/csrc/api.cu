@@ -73,6 +73,7 @@ ob_status make_ctx(void* stream, LaunchCtx* c) {
   c->err = d.err;
   c->num_sms = d.num_sms;
   c->pdl = env_flag("OB_PDL", true);
+  c->l2_prefetch = env_flag("OB_L2_PREFETCH", true);
   return OB_OK;
 }
 
@@ -89,12 +90,17 @@ ob_status status_of(cudaError_t e) {
   return OB_ERR_CUDA;
 }
 
-ob_status run_sign_gemm(const SignGemmArgs& g, int path, const LaunchCtx& c) {
+ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) {
+  SignGemmArgs g = g_in;
+  g.l2_prefetch = (c.pdl && c.l2_prefetch) ? 1 : 0;
   // Measured on B200 (4096 x 4096 layer, one call per CUDA-graph node): one token is
   // fastest on the table-driven CUDA-core kernel, 2..16 tokens on the warp-level
-  // MMA kernel, more on the tcgen05 GEMM.
-  if (path == OB_PATH_AUTO)
+  // MMA kernel, more on the tcgen05 GEMM.  K beyond the tcgen05 GEMM's limit goes
+  // to the warp-level MMA kernel, 16 tokens per launch.
+  if (path == OB_PATH_AUTO) {
     path = g.M == 1 ? OB_PATH_SIMT : (g.M <= decode_max_m() ? OB_PATH_MMA_DECODE : OB_PATH_TC);
+    if (path == OB_PATH_TC && g.K > sign_gemm_tc_max_k()) path = OB_PATH_MMA_DECODE;
+  }
   cudaError_t e;
   switch (path) {
     case OB_PATH_SIMT: e = launch_sign_gemm_simt(g, c); break;

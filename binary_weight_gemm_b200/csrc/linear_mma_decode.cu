@@ -193,12 +193,12 @@ __global__ void __launch_bounds__(kThreads, 2) sign_gemm_mma_decode_kernel(SignG
     }
   };
 
-  pdl_launch_dependents();
-  // Weights and the output scale do not depend on the previous grid: fetch them first.
-  int64_t chunk = warp;
-  fetch_words(chunk, 0);
-  const int my_row = tid & (kRowsPerCta - 1);  // the output row this thread stores
-  const float osc = (n0 + my_row < g.R) ? __ldg(g.oscale + n0 + my_row) : 0.f;
+  // Before the previous grid has finished, only pull this CTA's sign rows (one
+  // contiguous block) into L2; the reads themselves come after pdl_wait.
+  if (g.l2_prefetch && warp == 0 && n0 < g.R) {
+    const int64_t rows = min64(kRowsPerCta, g.R - n0);
+    prefetch_block_l2(g.S + n0 * Wd, (uint64_t)(rows * Wd) * 4u, lane);
+  }
 
   constexpr int kSets = NN == 1 ? 4 : 2;  // independent accumulator chains
   float acc[kSets][kRowTiles][NN][4];
@@ -211,7 +211,12 @@ __global__ void __launch_bounds__(kThreads, 2) sign_gemm_mma_decode_kernel(SignG
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[q][rt][nn][i] = 0.f;
 
-  pdl_wait();  // activations (and the output) depend on the previous grid in the stream
+  pdl_wait();  // every input may have been written by the previous grid in the stream
+  pdl_launch_dependents();  // the next grid may start (one grid ahead at most)
+  int64_t chunk = warp;
+  fetch_words(chunk, 0);
+  const int my_row = tid & (kRowsPerCta - 1);  // the output row this thread stores
+  const float osc = (n0 + my_row < g.R) ? __ldg(g.oscale + n0 + my_row) : 0.f;
   int buf = 0;
   for (; chunk < nchunks; chunk += kWarps, buf ^= 1) {
     stage_x(chunk);
@@ -303,10 +308,7 @@ cudaError_t launch_tok(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c) {
   cfg.stream = c.stream;
   cudaLaunchAttribute attr[1];
   int na = 0;
-  // Programmatic dependent launch pays off only for the 16-token build here: for
-  // shorter calls the early-launched CTAs cost more than the overlap they buy
-  // (measured per call in a graph of back-to-back 4096 x 4096 layers).
-  if (c.pdl && TOK > 8) {
+  if (c.pdl) {
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     na = 1;

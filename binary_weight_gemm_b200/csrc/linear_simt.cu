@@ -30,6 +30,14 @@ template <int MT>
 __host__ __device__ constexpr int rows_per_warp() { return MT >= 4 ? 1 : (MT == 2 ? 2 : 4); }
 constexpr int kPitch = 33;  // 32 groups + 1: odd pitch
 
+// Programmatic dependent launch: every read of an input comes after pdl_wait, and
+// the next grid is released after it, so at most one grid waits ahead.  (No L2
+// prefetch of the weights here: on B200 it made these short kernels slower.)
+__device__ __forceinline__ void prologue_wait() {
+  pdl_wait();
+  pdl_launch_dependents();
+}
+
 template <int MT, int Q>
 __global__ void __launch_bounds__(kSimtThreads) sign_gemv_simt_kernel(SignGemmArgs g, int64_t m0) {
   constexpr int kRowsPerWarp = rows_per_warp<MT>();
@@ -42,6 +50,7 @@ __global__ void __launch_bounds__(kSimtThreads) sign_gemv_simt_kernel(SignGemmAr
   const int64_t G = (Wd + Q - 1) / Q;     // groups per row (Q = 4 only when Wd % 4 == 0)
   const int64_t mt = min64(MT, g.M - m0);
   const int64_t row0 = (int64_t)blockIdx.x * kRowsPerCta + warp * kRowsPerWarp;
+  prologue_wait();
 
   float acc[kRowsPerWarp][MT];
 #pragma unroll
@@ -166,6 +175,7 @@ __global__ void __launch_bounds__(kSimtThreads) sign_gemv_lut_kernel(SignGemmArg
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t K = g.K, Wd = K / 32, G = (Wd + Q - 1) / Q;
   const int64_t row0 = (int64_t)blockIdx.x * kRowsPerCta + warp * kRowsPerWarp;
+  prologue_wait();
   float acc[kRowsPerWarp];
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) acc[r] = 0.f;
@@ -258,6 +268,26 @@ __global__ void __launch_bounds__(kSimtThreads) sign_gemv_lut_kernel(SignGemmArg
   }
 }
 
+// Launch with programmatic stream serialization when enabled: the kernel may
+// start while the previous grid in the stream is still running.
+template <typename Kern>
+cudaError_t launch_pdl(Kern kern, int64_t blocks, size_t smem, const SignGemmArgs& g, int64_t m0,
+                       const LaunchCtx& c) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+  cfg.blockDim = dim3(kSimtThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = c.pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, g, m0);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int Q>
 cudaError_t launch_lut(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c) {
   const size_t smem = sizeof(float) * 16 * 32 * Q * 8;
@@ -267,9 +297,7 @@ cudaError_t launch_lut(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c) {
     if (e != cudaSuccess) return e;
   }
   constexpr int kRowsPerCta = kSimtWarps * 4;
-  const unsigned blocks = (unsigned)((g.R + kRowsPerCta - 1) / kRowsPerCta);
-  kern<<<blocks, kSimtThreads, smem, c.stream>>>(g, m0);
-  return cudaGetLastError();
+  return launch_pdl(kern, (g.R + kRowsPerCta - 1) / kRowsPerCta, smem, g, m0, c);
 }
 
 template <int MT, int Q>
@@ -281,9 +309,7 @@ cudaError_t launch_one(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c) {
     if (e != cudaSuccess) return e;
   }
   constexpr int kRowsPerCta = kSimtWarps * rows_per_warp<MT>();
-  const unsigned blocks = (unsigned)((g.R + kRowsPerCta - 1) / kRowsPerCta);
-  kern<<<blocks, kSimtThreads, smem, c.stream>>>(g, m0);
-  return cudaGetLastError();
+  return launch_pdl(kern, (g.R + kRowsPerCta - 1) / kRowsPerCta, smem, g, m0, c);
 }
 
 }  // namespace

@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     sh->abort_flag = 0;
     fence_mbar_init();
   }
+  pdl_wait();  // every input may have been written by the previous grid in the stream
   // Input-scale pairs as bf16x2 (round to nearest even); ones without a scale.
   for (int64_t i = tid; i < (K + 1) / 2; i += kThreads) {
     const float lo = g.iscale ? __ldg(g.iscale + 2 * i) : 1.f;
@@ -205,7 +206,6 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     const int half = (warp - 4) >> 2;     // which half of the token columns
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int c0 = half * (kTok / 64), c1 = c0 + kTok / 64;
-    pdl_wait();
     int64_t it = 0;
     if (tma_store) {
       // bf16 Y: the tile is staged in shared memory as [token][row], Y's own
@@ -321,8 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
-      pdl_wait();
-      int64_t gstage = 0;
+        int64_t gstage = 0;
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
         const int32_t m0 = (int32_t)((tile / n_blocks) * kTok);
@@ -413,6 +412,8 @@ EncodeTiledFn get_encode_fn() {
 }
 
 }  // namespace
+
+int64_t sign_gemm_tc_max_k() { return kMaxK; }
 
 cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
   if (g.M == 0 || g.R == 0 || g.K == 0) return cudaSuccess;

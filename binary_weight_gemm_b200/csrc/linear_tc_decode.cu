@@ -119,7 +119,18 @@ __global__ void __launch_bounds__(kThreads, 2) sign_gemm_tc_decode_kernel(SignGe
   const int64_t n0 = (int64_t)blockIdx.y * kRows;
   const int64_t mt = min64(kTok, g.M - m0);
 
-  // Row threads request their packed words first: they depend on nothing.
+  // Before the previous grid has finished: only L2 prefetches of this CTA's rows.
+  if (g.l2_prefetch && warp == 0 && n0 < g.R) {
+    const int64_t rows = min64(kRows, g.R - n0);
+    const int64_t w_lo = (int64_t)st0 * 2, w_hi = min64(Wd, (int64_t)st1 * 2);
+    if ((Wd & 3) == 0 && (w_lo & 3) == 0) {  // 16-byte aligned row pieces
+      for (int64_t r = 0; r < rows; ++r)
+        if ((r & 31) == lane) prefetch_l2_bulk(g.S + (n0 + r) * Wd + w_lo, (uint32_t)((w_hi - w_lo) * 4));
+    }
+  }
+  pdl_wait();  // every input may have been written by the previous grid in the stream
+  pdl_launch_dependents();  // the next grid may start (one grid ahead at most)
+
   const int64_t n = n0 + (tid & 127);
   const bool row_ok = warp < 4 && n < g.R;
   const int64_t w_begin = (int64_t)st0 * 2;  // even
@@ -161,7 +172,6 @@ __global__ void __launch_bounds__(kThreads, 2) sign_gemm_tc_decode_kernel(SignGe
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
   volatile int* abort_flag = &sh->abort_flag;
-  pdl_launch_dependents();
 
   if (warp < 4) {
     // ------------------------------------------------ row threads
@@ -186,9 +196,6 @@ __global__ void __launch_bounds__(kThreads, 2) sign_gemm_tc_decode_kernel(SignGe
       for (int j = 0; j < kRing; ++j)
         if (j < nst) mbar_arrive(&sh->full[j]);
     }
-
-    // Activations depend on the previous grid in the stream.
-    pdl_wait();
 
     // X' = x ⊙ iscale into the swizzled B tile, in (i, i+16) pair order.
     // Unit = (token half h, stage j, word g, 8-column block cb): 8 tokens x 8 pairs.
@@ -324,7 +331,6 @@ __global__ void __launch_bounds__(kThreads, 2) sign_gemm_tc_decode_kernel(SignGe
       mma_commit(&sh->dfull);  // also covers abort: arrives once prior MMAs retire
     }
     __syncwarp();
-    pdl_wait();  // this warp stores Y in the cluster reduction below
   }
 
   if constexpr (kCluster) {

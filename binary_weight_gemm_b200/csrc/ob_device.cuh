@@ -175,7 +175,30 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
+// Prefetch [p, p + bytes) into L2 (a hint: no data reaches the thread and no
+// ordering is implied).  p must be 16-byte aligned; bytes is rounded down to a
+// multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  bytes &= ~15u;
+  if (bytes)
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
+
+// One warp prefetches a contiguous block into L2 in 4 KB pieces, one piece per lane
+// at a time.  base must be 16-byte aligned.
+__device__ __forceinline__ void prefetch_block_l2(const void* base, uint64_t bytes, int lane) {
+  const char* p = static_cast<const char*>(base);
+  for (uint64_t off = (uint64_t)lane * 4096u; off < bytes; off += 32u * 4096u)
+    prefetch_l2_bulk(p + off, (uint32_t)min64(4096, (int64_t)(bytes - off)));
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
+//
+// Rule for every kernel here: nothing is read from global memory before
+// pdl_wait() (the previous grid may have written any input, weights included);
+// what may run earlier is setup that touches no input and L2 prefetches, which
+// are hints.
 
 // Wait until the grids this launch depends on have completed and flushed memory.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -13,6 +13,7 @@ struct LaunchCtx {
   unsigned* err;   // device error word of the current device
   int num_sms;     // multiprocessors of the current device
   bool pdl;        // launch with programmatic stream serialization
+  bool l2_prefetch;  // with pdl: prefetch the weights into L2 before waiting on the previous grid
 };
 
 // One sign-product layer  Y[m, n] = oscale[n] * sum_k (x[m, k] * iscale[k]) * s[n, k],
@@ -29,6 +30,7 @@ struct SignGemmArgs {
   void* Y;
   int64_t ldy;
   int y_dtype;          // ob_out_dtype
+  int l2_prefetch;      // set by the dispatcher: prefetch this launch's weights into L2 first
 };
 
 cudaError_t launch_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* out, const LaunchCtx& c);
@@ -37,6 +39,8 @@ cudaError_t launch_sign_gemm_simt(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_tc_decode(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_mma_decode(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c);
+// Largest K the tcgen05 GEMM takes (its input-scale pairs live in shared memory).
+int64_t sign_gemm_tc_max_k();
 
 // SVID power iteration pieces (see svid.cu).
 size_t svid_workspace_bytes(int64_t N, int64_t K);

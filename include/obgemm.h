@@ -71,7 +71,7 @@ typedef enum ob_status {
   OB_ERR_WORKSPACE = 6,       /* workspace NULL or smaller than required */
   OB_ERR_CUDA = 7,            /* a CUDA runtime call or kernel launch failed */
   OB_ERR_DEVICE_TIMEOUT = 8,  /* a bounded wait inside a kernel ran out */
-  OB_ERR_UNSUPPORTED = 9,     /* device is not sm_100 or an option is unknown */
+  OB_ERR_UNSUPPORTED = 9,     /* device is not sm_100, an option is unknown, or OB_PATH_TC with K > 32768 */
   OB_ERR_DEVICE_BOUNDS = 10   /* a kernel's own bounds check refused an access */
 } ob_status;
 
@@ -82,10 +82,10 @@ typedef enum ob_out_dtype {
 
 /* Kernel choice for ob_linear_ex / dbf_linear_ex. */
 typedef enum ob_path {
-  OB_PATH_AUTO = 0,        /* M == 1: OB_PATH_SIMT; M <= 16: OB_PATH_MMA_DECODE; else OB_PATH_TC */
+  OB_PATH_AUTO = 0,        /* M == 1: OB_PATH_SIMT; M <= 16 or K > 32768: OB_PATH_MMA_DECODE; else OB_PATH_TC */
   OB_PATH_SIMT = 1,        /* CUDA-core select/add mat-vec (any M; slow for M > 4) */
   OB_PATH_TC_DECODE = 2,   /* tcgen05, signs unpacked into tensor memory, M <= 16 per pass */
-  OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA) */
+  OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA); K <= 32768 */
   OB_PATH_MMA_DECODE = 4   /* warp-level MMA, signs unpacked in registers, M <= 16 per pass */
 } ob_path;
 

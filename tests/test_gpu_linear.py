@@ -58,6 +58,7 @@ SHAPES = [  # (M, N, K)
     (17, 130, 160),    # M over one decode pass
     (300, 260, 192),   # ragged M and N tiles for the large-M kernel
     (513, 128, 4096),
+    (300, 264, 192),   # ragged M and N, Y rows 16-byte aligned (TMA-stored output tile)
 ]
 
 
@@ -129,6 +130,29 @@ def test_linear_end_to_end_pipeline_vs_oracle_pipeline(ops):
     for path in PATHS.values():
         Y = ops.ob_linear(_x_bf16(xb), P, a_g, b_g, path=path)
         assert_gemm_close(Y, ref, what=f"pipeline path {path}")
+
+
+@pytest.mark.parametrize("M,K,path", [(260, 20480, "tc"), (40, 20480, "auto"), (20, 36864, "auto")])
+def test_linear_long_k(ops, M, K, path):
+    # K past 16384 runs the three-stage tcgen05 kernel; past 32768 AUTO takes the
+    # warp-level MMA kernel in 16-token launches.
+    N = 136
+    seed = K + M
+    W = synth.weights(seed, N, K)
+    a, b, _ = oracle.svid_rank1(W)
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    xb, x = synth.activations(seed, M, K)
+    Y = _run(ops, xb, W, a, b, PATHS.get(path, 0))
+    assert_gemm_close(Y, _ref(x, W, a, b), what=f"long K {M}x{N}x{K} {path}")
+
+
+def test_tc_path_rejects_k_beyond_limit(ops):
+    from binary_weight_gemm_b200._lib import ObError
+    K = 32768 + 32
+    X = torch.zeros((32, K), dtype=torch.bfloat16, device="cuda")
+    P = torch.zeros((128, K // 32), dtype=torch.int32, device="cuda")
+    with pytest.raises(ObError):
+        ops.ob_linear(X, P, torch.ones(128, device="cuda"), torch.ones(K, device="cuda"), path=PATHS["tc"])
 
 
 def test_linear_degenerate_sizes(ops):
