@@ -539,6 +539,118 @@ def run_prefill(args, world, rank, local):
         }
         print(json.dumps(line), flush=True)
 
+STACK_SHAPES = {"q": (4096, 4096), "k": (4096, 4096), "v": (4096, 4096), "o": (4096, 4096),
+                "gate": (4096, 11008), "up": (4096, 11008), "down": (11008, 4096)}  # name: (K, N)
+
+
+def run_stack(args, world, rank, local):
+    """Decode through a stack of 7B-shaped OneBit linear layers, one token (batch M) at a time.
+
+    Per block: q, k, v, o (4096 -> 4096), gate, up (4096 -> 11008), down (11008 -> 4096),
+    chained through their outputs (q, k, v read the block input; o reads q's output;
+    gate and up read o's; down reads gate's; the next block reads down's).  Attention,
+    the gated activation and the norms are not part of this library, so a layer's output
+    feeds the next layer directly.  32 blocks = 224 distinct packed weight buffers (812 MB,
+    6.5 x L2).  One CUDA graph per token and batch size, programmatic dependent launch
+    between calls.
+    """
+    import torch
+    from binary_weight_gemm_b200 import build, synth
+    build.build()
+    from binary_weight_gemm_b200 import ops
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    peaks = load_peaks()
+    blocks = args.blocks
+    ms_list = (1, 16)
+    # One seeded matrix per shape, packed and SVID'd by the library, cloned into every block.
+    base = {}
+    for K, N in sorted(set(STACK_SHAPES.values())):
+        W = torch.from_numpy(synth.weights(7 + K % 97 + N % 89, N, K)).to(dev)
+        P = ops.ob_pack_signs(W, stream=stream)
+        a, b, _, _, _ = ops.ob_svid_rank1(W, stream=stream)
+        base[(K, N)] = (P, a, b)
+        del W
+    layers = [{name: tuple(t.clone() for t in base[STACK_SHAPES[name]]) for name in STACK_SHAPES}
+              for _ in range(blocks)]
+    wbytes = sum(N * K // 8 + 4 * (N + K) for K, N in STACK_SHAPES.values()) * blocks
+    acts = {}
+    for m in ms_list:
+        x0 = torch.from_numpy(synth.activations(7, m, 4096)[0].view(np.int16)).to(dev).view(torch.bfloat16)
+        buf = {name: torch.empty((m, N), dtype=torch.bfloat16, device=dev) for name, (K, N) in STACK_SHAPES.items()}
+        acts[m] = (x0, buf)
+
+    def token(m, s):
+        x0, buf = acts[m]
+        x = x0
+        for L in layers:
+            for name in ("q", "k", "v"):
+                P, a, b = L[name]
+                ops.ob_linear(x, P, a, b, out=buf[name], stream=s)
+            P, a, b = L["o"]
+            ops.ob_linear(buf["q"], P, a, b, out=buf["o"], stream=s)
+            for name in ("gate", "up"):
+                P, a, b = L[name]
+                ops.ob_linear(buf["o"], P, a, b, out=buf[name], stream=s)
+            P, a, b = L["down"]
+            ops.ob_linear(buf["gate"], P, a, b, out=buf["down"], stream=s)
+            x = buf["down"]
+
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for m in ms_list:
+            token(m, stream)
+        stream.synchronize()
+        for m in ms_list:
+            graphs[m] = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graphs[m], stream=stream):
+                token(m, stream)
+    calls = 7 * blocks
+
+    def step():
+        for m in ms_list:
+            graphs[m].replay()
+
+    ms_max, ms, clocks = _timed(step, args, world, stream, local)
+    per_m = {}
+    for m in ms_list:
+        reps = max(3, args.steps // 2)
+        with torch.cuda.stream(stream):
+            graphs[m].replay()
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                graphs[m].replay()
+            e1.record(stream)
+            stream.synchronize()
+        t_tok = e0.elapsed_time(e1) * 1e-3 / reps
+        abytes = sum(2 * m * (K + N) for K, N in STACK_SHAPES.values()) * blocks
+        per_m[str(m)] = {"us_per_token": t_tok * 1e6, "tokens_per_s": m / t_tok,
+                         "weight_gbs": wbytes / t_tok / 1e9, "hbm_gbs": (wbytes + abytes) / t_tok / 1e9,
+                         "frac_hbm": (wbytes + abytes) / t_tok / 1e9 / peaks["hbm_gbs"],
+                         "us_per_call": t_tok * 1e6 / calls}
+    step_bytes_total = sum(wbytes + sum(2 * m * (K + N) for K, N in STACK_SHAPES.values()) * blocks
+                           for m in ms_list)
+    value = world * step_bytes_total * args.steps / (ms_max * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"onebit_decode_stack_7b_{blocks}blocks", "M": list(ms_list),
+                       "layers_per_token": calls, "weights_mb": wbytes / 1e6,
+                       "l2": f"inputs larger than L2: {blocks * 7} distinct weight buffers ({wbytes / 1e6:.0f} MB)",
+                       "graph": "one CUDA graph per token and M, programmatic dependent launch between calls",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "per_m": per_m,
+            "gpu_launches": args.steps * calls * len(ms_list), "clocks": clocks, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    graphs.clear()
+
+
 def _time_calls(fn, stream, reps):
     import torch
     with torch.cuda.stream(stream):
@@ -574,25 +686,31 @@ def run_extra(ops, dev, stream, peaks):
                                       "frac_bf16_sustained": fl / t / 1e12 / (peaks["bf16_tflops_sustained"] or 1),
                                       "kernel": "sign_gemm_tc_kernel"}
     del sets
-    # DBF: K = N = 4096, r = 2048.
-    f = synth.dbf_factors(3, 4096, 2048, 4096)
-    SB = ops.ob_pack_signs(torch.from_numpy(f["S_B"].astype(np.float32)).to(dev), stream=stream)
-    SA = ops.ob_pack_signs(torch.from_numpy(f["S_A"].astype(np.float32)).to(dev), stream=stream)
-    vec = {k: torch.from_numpy(f[k]).to(dev) for k in ("a", "m", "b")}
-    for M in (1, 512):
-        nset = 64 if M == 1 else 8
-        pool = [(SB.clone(), SA.clone()) for _ in range(nset)]
-        X = torch.from_numpy(synth.activations(3, M, 4096)[0].view(np.int16)).to(dev).view(torch.bfloat16)
-        Y = torch.empty((M, 4096), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(ops.dbf_workspace_size(M, 2048), dtype=torch.uint8, device=dev)
-        t = _time_calls(lambda i: ops.dbf_linear(X, pool[i % nset][0], vec["m"], pool[i % nset][1], vec["a"],
-                                                 vec["b"], out=Y, workspace=ws, stream=stream), stream,
-                        max(50, 4 * nset))
-        fl = 2 * M * 2048 * (4096 + 4096)
-        byts = 2048 * 4096 // 8 * 2 + 4 * (4096 * 2 + 2048) + 2 * M * 4096 * 2
-        out[f"dbf_M{M}"] = {"us_per_call": t * 1e6, "tflops_equiv": fl / t / 1e12, "hbm_gbs": byts / t / 1e9,
-                            "frac_hbm": byts / t / 1e9 / peaks["hbm_gbs"],
-                            "frac_bf16_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
+    # DBF: K = N = 4096, r = 2048 (the configured workload) and the middle dimensions of
+    # about 0.5, 1.5 and 2.3 bits per weight (non-uniform r per layer).
+    for r in (2048, 1056, 3072, 4704):
+        f = synth.dbf_factors(3, 4096, r, 4096)
+        SB = ops.ob_pack_signs(torch.from_numpy(f["S_B"].astype(np.float32)).to(dev), stream=stream)
+        SA = ops.ob_pack_signs(torch.from_numpy(f["S_A"].astype(np.float32)).to(dev), stream=stream)
+        vec = {k: torch.from_numpy(f[k]).to(dev) for k in ("a", "m", "b")}
+        wbytes = r * 4096 // 8 * 2
+        for M in (1, 512):
+            nset = max(8, -(-3 * 126 * 2**20 // (wbytes + 2 * M * 4096 * 2)))  # > 3x L2 in total
+            pool = [(SB.clone(), SA.clone()) for _ in range(nset)]
+            X = torch.from_numpy(synth.activations(3, M, 4096)[0].view(np.int16)).to(dev).view(torch.bfloat16)
+            Y = torch.empty((M, 4096), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(ops.dbf_workspace_size(M, r), dtype=torch.uint8, device=dev)
+            t = _time_calls(lambda i: ops.dbf_linear(X, pool[i % nset][0], vec["m"], pool[i % nset][1], vec["a"],
+                                                     vec["b"], out=Y, workspace=ws, stream=stream), stream,
+                            max(50, 2 * nset))
+            fl = 2 * M * r * (4096 + 4096)
+            byts = wbytes + 4 * (4096 * 2 + r) + 2 * M * 4096 * 2
+            key = f"dbf_M{M}" if r == 2048 else f"dbf_r{r}_M{M}"
+            out[key] = {"us_per_call": t * 1e6, "r": r, "bits_per_weight": r * 8192 / 4096**2,
+                        "tflops_equiv": 2 * M * 4096 * 4096 / t / 1e12, "tflops_alg": fl / t / 1e12,
+                        "hbm_gbs": byts / t / 1e9, "frac_hbm": byts / t / 1e9 / peaks["hbm_gbs"],
+                        "frac_bf16_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
+            del pool
     return out
 
 
@@ -602,8 +720,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
-                    help="decode: OneBit 4096x4096 at M=1,4,16 (default); prefill: M=2048, 4096 -> 11008")
+    ap.add_argument("--workload", choices=["decode", "prefill", "stack"], default="decode",
+                    help="decode: OneBit 4096x4096 at M=1,4,16 (default); prefill: M=2048, 4096 -> 11008; "
+                         "stack: one token through 32 blocks of 7B-shaped OneBit layers at M=1 and 16")
+    ap.add_argument("--blocks", type=int, default=32, help="blocks of the stack workload")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-extra", dest="extra", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -616,6 +736,8 @@ def main():
             run_reference(args, world, rank)
         elif args.workload == "prefill":
             run_prefill(args, world, rank, local)
+        elif args.workload == "stack":
+            run_stack(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -10,7 +10,8 @@ Everything is plain NumPy in float64, written from the definitions on the pages:
 
 * OneBit, from "1bit量化" (blog.zerodtree.com, notes on "OneBit: Towards
   Extremely Low-bit Large Language Models"): sign/value split and rank-1 SVID
-  (section "rank-1 approximation"), Proposition 1, Lemma 1, Proposition 2.
+  (section "rank-1 approximation"), Proposition 1, Lemma 1, Proposition 2, and
+  the LayerNorm that follows the layer (knowledge-distillation section).
 * DBF, from "Addition is almost all you need: Compressing large language models
   with double binary factorization" (gist.science, section "Methodologie:
   Double Binary Factorization (DBF)"): the factorised weight and its inference
@@ -27,11 +28,12 @@ Parity status: every public function here is pinned by tests under
 """
 from .onebit import (sign_pm1, pack_signs, unpack_signs, rank1_svd, svid_rank1,
                      onebit_weight, onebit_linear, onebit_linear_packed,
-                     onebit_linear_prop1)
+                     onebit_linear_prop1, layernorm, onebit_linear_ln, LN_EPS)
 from .dbf import dbf_weight, dbf_linear, dbf_linear_chain
 
 __all__ = [
     "sign_pm1", "pack_signs", "unpack_signs", "rank1_svd", "svid_rank1",
     "onebit_weight", "onebit_linear", "onebit_linear_packed", "onebit_linear_prop1",
+    "layernorm", "onebit_linear_ln", "LN_EPS",
     "dbf_weight", "dbf_linear", "dbf_linear_chain",
 ]

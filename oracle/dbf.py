@@ -39,7 +39,9 @@ def dbf_linear(X, S_A, S_B, a, m, b) -> np.ndarray:
 def dbf_linear_chain(X, S_A, S_B, a, m, b) -> np.ndarray:
     """The page's inference order ((((X ⊙ b^T) S_B^T) ⊙ m^T) S_A^T) ⊙ a^T, float64.
 
-    Used only to check the chain against the direct form.
+    Equal to the direct form in exact arithmetic (pinned by the tests against
+    dbf_linear); the GPU parity tests use it where r and K are large enough that
+    materialising W_hat would cost seconds per case.
     """
     X = np.asarray(X, dtype=np.float64)
     T = (X * np.asarray(b, dtype=np.float64)[None, :]) @ np.asarray(S_B, dtype=np.float64).T

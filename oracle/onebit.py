@@ -115,3 +115,25 @@ def onebit_linear_prop1(X: np.ndarray, S: np.ndarray, a: np.ndarray, b: np.ndarr
     X = np.asarray(X, dtype=np.float64)
     Xb = X * np.asarray(b, dtype=np.float64)[None, :]
     return (Xb @ np.asarray(S, dtype=np.float64).T) * np.asarray(a, dtype=np.float64)[None, :]
+
+
+# Layer normalisation after the OneBit layer ("1bit量化", knowledge-distillation
+# section: the student computes Y with Proposition 1 and then Z = LayerNorm(Y)).
+# Reading (the page gives the name only): per token, i.e. per row of Y, over its
+# N features; the biased variance; eps = 1e-5 inside the square root; no affine
+# parameters (the page shows none).
+LN_EPS = 1e-5
+
+
+def layernorm(Y: np.ndarray, eps: float = LN_EPS) -> np.ndarray:
+    """Z[m, :] = (Y[m, :] - mean) / sqrt(var + eps), mean and biased var over the row, fp64."""
+    Y = np.asarray(Y, dtype=np.float64)
+    mean = Y.mean(axis=1, keepdims=True)
+    var = ((Y - mean) ** 2).mean(axis=1, keepdims=True)
+    return (Y - mean) / np.sqrt(var + eps)
+
+
+def onebit_linear_ln(X: np.ndarray, S: np.ndarray, a: np.ndarray, b: np.ndarray,
+                     eps: float = LN_EPS) -> np.ndarray:
+    """Z = LayerNorm(Y) with Y the OneBit layer in the direct form."""
+    return layernorm(onebit_linear(X, S, a, b), eps)

@@ -57,6 +57,18 @@ def test_dbf_workload_full(ops, M):
     assert_gemm_close(Y, _ref(x, f), what=f"dbf workload M={M}")
 
 
+# Middle dimensions for about 0.5, 1.5, 1.8 and 2.3 bits per weight at K = N = 4096
+# (bits ~ r (K + N) / (N K)): non-uniform r per layer, with tile tails in both sign GEMMs.
+@pytest.mark.parametrize("r", [1056, 3072, 3680, 4704])
+@pytest.mark.parametrize("M", [1, 16, 300])
+def test_dbf_general_r(ops, r, M):
+    f = synth.dbf_factors(r + M, 4096, r, 4096)
+    xb, x = synth.activations(r, M, 4096)
+    Y = _run(ops, xb, f, PATHS["auto"])
+    ref = oracle.dbf_linear_chain(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"])
+    assert_gemm_close(Y, ref, what=f"dbf r={r} M={M}")
+
+
 def test_dbf_fp32_output(ops):
     # Smallest middle dimension (one packed word per S_A row), fp32 output.
     f = synth.dbf_factors(11, 256, 32, 256)

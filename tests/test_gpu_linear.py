@@ -227,3 +227,46 @@ def test_cuda_graph_replay_matches(ops):
     g.replay()
     torch.cuda.synchronize()
     assert_gemm_close(Y, _ref(x, W, a, b), what="graph replay")
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 40])
+def test_chained_layers_in_graph(ops, M):
+    # Eight 512 x 512 layers chained through their outputs (layer i+1 reads layer i's Y),
+    # captured in one CUDA graph; calls may launch before their predecessor has finished
+    # (programmatic dependent launch), so each must read its input only after it is complete.
+    # Every layer is checked against the oracle on the bf16 input it actually received.
+    K = 512
+    layers = []
+    for i in range(8):
+        W = synth.weights(100 + i, K, K)
+        a, b, _ = oracle.svid_rank1(W)
+        layers.append((W, a.astype(np.float32), b.astype(np.float32)))
+    dev = [(ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b)) for W, a, b in layers]
+    xb, _ = synth.activations(100, M, K)
+    X = _x_bf16(xb)
+    Ys = [torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for _ in layers]
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+
+    def chain():
+        x = X
+        for (P, a, b), Y in zip(dev, Ys):
+            ops.ob_linear(x, P, a, b, out=Y, stream=s)
+            x = Y
+
+    with torch.cuda.stream(s):
+        chain()  # warm up outside capture
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            chain()
+    for Y in Ys:
+        Y.zero_()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    x_in = X.float().cpu().numpy().astype(np.float64)
+    for i, ((W, a, b), Y) in enumerate(zip(layers, Ys)):
+        assert_gemm_close(Y, _ref(x_in, W, a, b), what=f"chained layer {i} M={M}")
+        x_in = Y.float().cpu().numpy().astype(np.float64)

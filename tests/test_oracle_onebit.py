@@ -291,3 +291,46 @@ def test_linear_packed_equals_unpacked():
     y1 = oracle.onebit_linear_packed(x, oracle.pack_signs(W), a, b)
     y2 = oracle.onebit_linear(x, oracle.sign_pm1(W), a, b)
     np.testing.assert_array_equal(y1, y2)
+
+
+# ---------------------------------------------------------------- LayerNorm after the layer
+
+def test_layernorm_golden(golden):
+    g = golden("layernorm_4.json")
+    np.testing.assert_allclose(oracle.layernorm(np.array(g["Y"]), eps=g["eps"]), np.array(g["Z"]),
+                               rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("M,N", [(1, 2), (3, 7), (16, 4096), (5, 11008)])
+def test_layernorm_matches_torch(M, N):
+    import torch
+    Y = np.random.default_rng(M * N).standard_normal((M, N)) * 3.0 + 0.7
+    ref = torch.nn.functional.layer_norm(torch.from_numpy(Y), (N,), eps=1e-5).numpy()
+    np.testing.assert_allclose(oracle.layernorm(Y, eps=1e-5), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_layernorm_invariants():
+    rng = np.random.default_rng(3)
+    Y = rng.standard_normal((6, 300)) * rng.uniform(0.1, 10, (6, 1)) + rng.uniform(-5, 5, (6, 1))
+    var = Y.var(axis=1)
+    Z = oracle.layernorm(Y, eps=1e-5)
+    np.testing.assert_allclose(Z.mean(axis=1), 0.0, atol=1e-13)
+    np.testing.assert_allclose(Z.var(axis=1), var / (var + 1e-5), rtol=1e-12)
+    # eps = 0: invariant under a positive per-row scale and a per-row shift.
+    alpha, beta = rng.uniform(0.5, 4, (6, 1)), rng.uniform(-3, 3, (6, 1))
+    np.testing.assert_allclose(oracle.layernorm(alpha * Y + beta, eps=0.0), oracle.layernorm(Y, eps=0.0),
+                               rtol=1e-10, atol=1e-12)
+
+
+def test_layernorm_degenerate_rows():
+    # One feature, or a constant row: y - mean = 0 everywhere, so Z = 0.
+    assert not oracle.layernorm(np.array([[3.0], [-2.0]])).any()
+    assert not oracle.layernorm(np.full((2, 5), 7.25)).any()
+
+
+def test_onebit_linear_ln_golden(golden):
+    # The 2 x 2 worked example gives Y = [-18, -57]: LayerNorm over two features is +/-1
+    # up to eps (mean -37.5, variance 19.5^2).
+    g = golden("onebit_linear_2x2.json")
+    Z = oracle.onebit_linear_ln(np.array(g["X"]), np.array(g["S"]), np.array(g["a"]), np.array(g["b"]))
+    np.testing.assert_allclose(Z, [[1.0, -1.0]], rtol=1e-7)
