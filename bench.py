@@ -685,7 +685,27 @@ def run_extra(ops, dev, stream, peaks):
                                       "frac_bf16_burst": fl / t / 1e12 / peaks["bf16_tflops"],
                                       "frac_bf16_sustained": fl / t / 1e12 / (peaks["bf16_tflops_sustained"] or 1),
                                       "kernel": "sign_gemm_tc_kernel"}
+    # The same prefill followed by LayerNorm over each token's outputs (ob_linear_ln).
+    t_ln = _time_calls(lambda i: ops.ob_linear_ln(sets[i % 3][0], sets[i % 3][1], a, b, out=sets[i % 3][2],
+                                                  stream=stream), stream, 30)
+    out["prefill_ln_2048x4096x11008"] = {"us_per_call": t_ln * 1e6, "tflops": fl / t_ln / 1e12,
+                                         "ln_us": (t_ln - t) * 1e6,
+                                         "kernels": "sign_gemm_tc_kernel + layernorm_rows_kernel"}
     del sets
+    # OneBit decode 4096 x 4096 followed by LayerNorm, M = 1 and 16 (pool of weight sets > L2).
+    W = torch.from_numpy(synth.weights(1, 4096, 4096)).to(dev)
+    P1 = ops.ob_pack_signs(W, stream=stream)
+    a1, b1, _, _, _ = ops.ob_svid_rank1(W, stream=stream)
+    del W
+    pool = [P1.clone() for _ in range(192)]
+    for M in (1, 16):
+        X = torch.from_numpy(synth.activations(1, M, 4096)[0].view(np.int16)).to(dev).view(torch.bfloat16)
+        Y = torch.empty((M, 4096), dtype=torch.bfloat16, device=dev)
+        t0 = _time_calls(lambda i: ops.ob_linear(X, pool[i % 192], a1, b1, out=Y, stream=stream), stream, 384)
+        t1 = _time_calls(lambda i: ops.ob_linear_ln(X, pool[i % 192], a1, b1, out=Y, stream=stream), stream, 384)
+        out[f"decode_ln_M{M}"] = {"us_per_call": t1 * 1e6, "linear_only_us": t0 * 1e6, "ln_us": (t1 - t0) * 1e6,
+                                  "hbm_gbs": decode_call_bytes(M) / t1 / 1e9}
+    del pool
     # DBF: K = N = 4096, r = 2048 (the configured workload) and the middle dimensions of
     # about 0.5, 1.5 and 2.3 bits per weight (non-uniform r per layer).
     for r in (2048, 1056, 3072, 4704):

@@ -31,6 +31,7 @@ SIGNATURES = {
     "ob_svid_rank1": (_I, [_P, _I64, _I64, _P, _P, _P, _I, _F, ctypes.POINTER(ctypes.c_int), _P, _SZ, _P]),
     "ob_linear": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _P]),
     "ob_linear_ex": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _I, _P]),
+    "ob_linear_ln": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _F, _I, _P]),
     "dbf_workspace_size": (_SZ, [_I64, _I64]),
     "dbf_linear": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P, _P, _I, _P, _SZ, _P]),
     "dbf_linear_ex": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P, _P, _I, _P, _SZ, _I, _P]),

@@ -214,6 +214,18 @@ ob_status ob_linear(const void* X, int64_t M, int64_t K, const uint32_t* W_packe
   return ob_linear_ex(X, M, K, W_packed, N, a, b, Y, y_dtype, OB_PATH_AUTO, stream);
 }
 
+ob_status ob_linear_ln(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,
+                       const float* b, void* Z, int z_dtype, float eps, int path, void* stream) {
+  if (!(eps >= 0.f) || eps > 3.0e38f) return OB_ERR_UNSUPPORTED;  // negative, NaN or infinite
+  if (M > 2147483647) return OB_ERR_SHAPE;                         // one CTA per row
+  ob_status st = ob_linear_ex(X, M, K, W_packed, N, a, b, Z, z_dtype, path, stream);
+  if (st != OB_OK || M == 0 || N == 0) return st;
+  LaunchCtx c;
+  st = make_ctx(stream, &c);
+  if (st != OB_OK) return st;
+  return launch_layernorm_rows(Z, M, N, N, z_dtype, eps, c) == cudaSuccess ? OB_OK : OB_ERR_CUDA;
+}
+
 size_t dbf_workspace_size(int64_t M, int64_t r) {
   if (M < 0 || r < 0) return 0;
   return align256((size_t)M * (size_t)r * 2);

@@ -49,6 +49,10 @@ ob_status run_svid(const float* W, int64_t N, int64_t K, float* a, float* b, flo
 
 cudaError_t launch_timeout_selftest(uint64_t limit_ns, const LaunchCtx& c);
 
+// Z = LayerNorm(Y) per row of the M x N matrix Y (row stride ld elements), in place.
+cudaError_t launch_layernorm_rows(void* Y, int64_t M, int64_t N, int64_t ld, int y_dtype, float eps,
+                                  const LaunchCtx& c);
+
 // Largest M handled by one pass of the tensor-memory decode kernel.
 constexpr int kDecodeMaxM = 16;
 

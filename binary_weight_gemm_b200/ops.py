@@ -109,6 +109,25 @@ def ob_linear(X: torch.Tensor, W_packed: torch.Tensor, a: torch.Tensor, b: torch
     return out
 
 
+def ob_linear_ln(X: torch.Tensor, W_packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor, eps: float = 1e-5,
+                 out_dtype: torch.dtype = torch.bfloat16, path: int = OB_PATH_AUTO, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """OneBit layer then LayerNorm over each token's N outputs: Z = LayerNorm(Y), no affine, biased variance."""
+    M, K = X.shape
+    N = W_packed.shape[0]
+    _need(X, "X", torch.bfloat16)
+    _need(W_packed, "W_packed", torch.int32, (N, K // 32))
+    _need(a, "a", torch.float32, (N,))
+    _need(b, "b", torch.float32, (K,))
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    _need(out, "out", out_dtype, (M, N))
+    st = _lib.lib().ob_linear_ln(_ptr(X), M, K, _ptr(W_packed), N, _ptr(a), _ptr(b), _ptr(out),
+                                 _out_code(out_dtype), float(eps), int(path), _stream(stream))
+    _lib.check("ob_linear_ln", st)
+    return out
+
+
 def dbf_workspace_size(M: int, r: int) -> int:
     return int(_lib.lib().dbf_workspace_size(M, r))
 

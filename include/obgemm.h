@@ -163,6 +163,25 @@ OB_API ob_status ob_linear_ex(const void* X, int64_t M, int64_t K,
                        const float* a, const float* b,
                        void* Y, int y_dtype, int path, void* stream);
 
+/*
+ * OneBit layer followed by LayerNorm: Z = LayerNorm(Y), Y as in ob_linear
+ * ("1bit量化", knowledge-distillation section: the student's Y is followed by
+ * Z = LayerNorm(Y)).  Per token (a row of Y), over its N features:
+ * z = (y - mean) / sqrt(var + eps), var the biased variance, no affine parameters
+ * (the page shows none).
+ *   Z      device, M x N, bf16 or fp32 by z_dtype; Y is computed into Z and
+ *          normalised in place (a second kernel; statistics from the stored Y).
+ *   eps    >= 0 and finite (1e-5 is the usual choice); otherwise OB_ERR_UNSUPPORTED
+ *          before anything is launched.
+ *   path   kernel for the linear layer, as in ob_linear_ex.
+ * Other arguments and errors as ob_linear_ex.  Asynchronous.  A row with a single
+ * feature, or a constant row, normalises to zeros.
+ */
+OB_API ob_status ob_linear_ln(const void* X, int64_t M, int64_t K,
+                       const uint32_t* W_packed, int64_t N,
+                       const float* a, const float* b,
+                       void* Z, int z_dtype, float eps, int path, void* stream);
+
 /* Bytes of device workspace dbf_linear needs (holds the M x r intermediate). */
 OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
 
