@@ -550,9 +550,10 @@ def run_stack(args, world, rank, local):
     chained through their outputs (q, k, v read the block input; o reads q's output;
     gate and up read o's; down reads gate's; the next block reads down's).  Attention,
     the gated activation and the norms are not part of this library, so a layer's output
-    feeds the next layer directly.  32 blocks = 224 distinct packed weight buffers (812 MB,
-    6.5 x L2).  One CUDA graph per token and batch size, programmatic dependent launch
-    between calls.
+    feeds the next layer directly.  32 blocks = 224 distinct packed weight buffers (819 MB,
+    6.5 x L2).  Timed: one ob_linear_stack per token (one persistent launch, grid barriers
+    where a layer reads an earlier output), captured as a CUDA graph per batch size; the
+    same token as 224 ob_linear calls in a graph is timed beside it.
     """
     import torch
     from binary_weight_gemm_b200 import build, synth
@@ -597,40 +598,67 @@ def run_stack(args, world, rank, local):
             ops.ob_linear(buf["gate"], P, a, b, out=buf["down"], stream=s)
             x = buf["down"]
 
-    graphs = {}
+    def spec(m):
+        """The same token as ob_linear_stack descriptors (after_previous where a layer reads an
+        output of the block it is in, or of the previous block)."""
+        x0, buf = acts[m]
+        out, x = [], x0
+        for bi, L in enumerate(layers):
+            for name in ("q", "k", "v"):
+                P, a, b = L[name]
+                out.append((x, P, a, b, buf[name], bi > 0 and name == "q"))
+            P, a, b = L["o"]
+            out.append((buf["q"], P, a, b, buf["o"], True))
+            for name in ("gate", "up"):
+                P, a, b = L[name]
+                out.append((buf["o"], P, a, b, buf[name], name == "gate"))
+            P, a, b = L["down"]
+            out.append((buf["gate"], P, a, b, buf["down"], True))
+            x = buf["down"]
+        return out
+
+    specs = {m: spec(m) for m in ms_list}
+    ws = torch.zeros(ops.ob_stack_workspace_size(), dtype=torch.uint8, device=dev)
+    graphs, pgraphs = {}, {}
     with torch.cuda.stream(stream):
         for m in ms_list:
             token(m, stream)
+            ops.ob_linear_stack(specs[m], m, workspace=ws, stream=stream)
         stream.synchronize()
         for m in ms_list:
             graphs[m] = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graphs[m], stream=stream):
                 token(m, stream)
+            pgraphs[m] = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(pgraphs[m], stream=stream):
+                ops.ob_linear_stack(specs[m], m, workspace=ws, stream=stream)
     calls = 7 * blocks
 
     def step():
         for m in ms_list:
-            graphs[m].replay()
+            pgraphs[m].replay()
 
     ms_max, ms, clocks = _timed(step, args, world, stream, local)
     per_m = {}
-    for m in ms_list:
-        reps = max(3, args.steps // 2)
-        with torch.cuda.stream(stream):
-            graphs[m].replay()
-            stream.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(reps):
-                graphs[m].replay()
-            e1.record(stream)
-            stream.synchronize()
-        t_tok = e0.elapsed_time(e1) * 1e-3 / reps
-        abytes = sum(2 * m * (K + N) for K, N in STACK_SHAPES.values()) * blocks
-        per_m[str(m)] = {"us_per_token": t_tok * 1e6, "tokens_per_s": m / t_tok,
-                         "weight_gbs": wbytes / t_tok / 1e9, "hbm_gbs": (wbytes + abytes) / t_tok / 1e9,
-                         "frac_hbm": (wbytes + abytes) / t_tok / 1e9 / peaks["hbm_gbs"],
-                         "us_per_call": t_tok * 1e6 / calls}
+    for mode, gs in (("persistent", pgraphs), ("per_call", graphs)):
+        for m in ms_list:
+            reps = max(3, args.steps // 2)
+            with torch.cuda.stream(stream):
+                gs[m].replay()
+                stream.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    gs[m].replay()
+                e1.record(stream)
+                stream.synchronize()
+            t_tok = e0.elapsed_time(e1) * 1e-3 / reps
+            abytes = sum(2 * m * (K + N) for K, N in STACK_SHAPES.values()) * blocks
+            per_m[f"{mode}_M{m}"] = {"us_per_token": t_tok * 1e6, "tokens_per_s": m / t_tok,
+                                     "weight_gbs": wbytes / t_tok / 1e9, "hbm_gbs": (wbytes + abytes) / t_tok / 1e9,
+                                     "frac_hbm": (wbytes + abytes) / t_tok / 1e9 / peaks["hbm_gbs"],
+                                     "us_per_layer": t_tok * 1e6 / calls}
+    assert ops.ob_last_device_error() == 0
     step_bytes_total = sum(wbytes + sum(2 * m * (K + N) for K, N in STACK_SHAPES.values()) * blocks
                            for m in ms_list)
     value = world * step_bytes_total * args.steps / (ms_max * 1e-3) / 1e9
@@ -642,13 +670,16 @@ def run_stack(args, world, rank, local):
             "config": {"workload": f"onebit_decode_stack_7b_{blocks}blocks", "M": list(ms_list),
                        "layers_per_token": calls, "weights_mb": wbytes / 1e6,
                        "l2": f"inputs larger than L2: {blocks * 7} distinct weight buffers ({wbytes / 1e6:.0f} MB)",
-                       "graph": "one CUDA graph per token and M, programmatic dependent launch between calls",
+                       "graph": "one CUDA graph per token and M holding one ob_linear_stack (persistent, "
+                                "grid barriers between dependent layers); per_call_* times one ob_linear "
+                                "per layer in a graph with programmatic dependent launch",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "per_m": per_m,
-            "gpu_launches": args.steps * calls * len(ms_list), "clocks": clocks, "cpu_baseline": None,
+            "gpu_launches": args.steps * len(ms_list), "clocks": clocks, "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)
     graphs.clear()
+    pgraphs.clear()
 
 
 def _time_calls(fn, stream, reps):

@@ -19,6 +19,15 @@ STATUS_NAMES = {
 OB_OUT_BF16, OB_OUT_F32 = 0, 1
 OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC_DECODE, OB_PATH_TC, OB_PATH_MMA_DECODE = 0, 1, 2, 3, 4
 
+
+
+class ObLayer(ctypes.Structure):
+    """struct ob_layer (include/obgemm.h): one layer of ob_linear_stack."""
+    _fields_ = [("X", ctypes.c_void_p), ("W_packed", ctypes.c_void_p), ("a", ctypes.c_void_p),
+                ("b", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("K", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("y_dtype", ctypes.c_int32), ("after_previous", ctypes.c_int32)]
+
+
 # Every function the header declares, with (restype, argtypes).
 _P, _I64, _I, _F, _SZ, _U64 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,
                                 ctypes.c_size_t, ctypes.c_uint64)
@@ -32,6 +41,8 @@ SIGNATURES = {
     "ob_linear": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _P]),
     "ob_linear_ex": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _I, _P]),
     "ob_linear_ln": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _F, _I, _P]),
+    "ob_stack_workspace_size": (_SZ, []),
+    "ob_linear_stack": (_I, [ctypes.POINTER(ObLayer), _I, _I64, _P, _SZ, _P]),
     "dbf_workspace_size": (_SZ, [_I64, _I64]),
     "dbf_linear": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P, _P, _I, _P, _SZ, _P]),
     "dbf_linear_ex": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P, _P, _I, _P, _SZ, _I, _P]),

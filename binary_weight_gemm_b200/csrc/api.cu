@@ -5,6 +5,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "ob_device.cuh"
 #include "ob_internal.h"
@@ -224,6 +225,33 @@ ob_status ob_linear_ln(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
   st = make_ctx(stream, &c);
   if (st != OB_OK) return st;
   return launch_layernorm_rows(Z, M, N, N, z_dtype, eps, c) == cudaSuccess ? OB_OK : OB_ERR_CUDA;
+}
+
+size_t ob_stack_workspace_size(void) { return 256; }
+
+ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  if (n_layers < 0 || M < 0 || M > kDecodeMaxM) return OB_ERR_SHAPE;
+  if (n_layers == 0 || M == 0) return OB_OK;
+  if (!layers) return OB_ERR_NULL;
+  if (!workspace) return OB_ERR_NULL;
+  if (misaligned(workspace)) return OB_ERR_ALIGN;
+  if (ws_bytes < ob_stack_workspace_size()) return OB_ERR_WORKSPACE;
+  std::vector<StackLayerHost> host((size_t)n_layers);
+  for (int i = 0; i < n_layers; ++i) {
+    const ob_layer& L = layers[i];
+    if (L.K < 32 || L.K % 32 != 0 || L.N < 1 || L.N > ((int64_t)1 << 35)) return OB_ERR_SHAPE;
+    if (L.y_dtype != OB_OUT_BF16 && L.y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
+    if (!L.X || !L.W_packed || !L.a || !L.Y) return OB_ERR_NULL;
+    if (misaligned(L.X) || misaligned(L.W_packed) || misaligned(L.a) || misaligned(L.Y) ||
+        (L.b && misaligned(L.b)))
+      return OB_ERR_ALIGN;
+    host[i] = StackLayerHost{L.X, L.W_packed, L.b, L.a, L.Y, L.K, L.N, L.y_dtype, L.after_previous ? 1 : 0};
+  }
+  LaunchCtx c;
+  ob_status st = make_ctx(stream, &c);
+  if (st != OB_OK) return st;
+  return status_of(launch_sign_stack(host.data(), n_layers, M, static_cast<unsigned*>(workspace), c));
 }
 
 size_t dbf_workspace_size(int64_t M, int64_t r) {

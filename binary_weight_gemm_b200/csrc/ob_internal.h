@@ -49,6 +49,22 @@ ob_status run_svid(const float* W, int64_t N, int64_t K, float* a, float* b, flo
 
 cudaError_t launch_timeout_selftest(uint64_t limit_ns, const LaunchCtx& c);
 
+// One layer of a persistent layer-stack launch (linear_stack.cu).
+struct StackLayerHost {
+  const void* X;        // bf16 [M, K]
+  const uint32_t* S;    // packed [N, K/32]
+  const float* iscale;  // [K] or null
+  const float* oscale;  // [N]
+  void* Y;              // [M, N]
+  int64_t K, N;
+  int y_dtype;
+  int barrier;          // reads an output of an earlier layer of the list
+};
+// Runs the list (M <= 16) as cooperative launches of at most stack_max_layers_per_launch()
+// layers; bar: 8 bytes of device memory (zeroed by the launcher).
+cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c);
+int stack_max_layers_per_launch();
+
 // Z = LayerNorm(Y) per row of the M x N matrix Y (row stride ld elements), in place.
 cudaError_t launch_layernorm_rows(void* Y, int64_t M, int64_t N, int64_t ld, int y_dtype, float eps,
                                   const LaunchCtx& c);

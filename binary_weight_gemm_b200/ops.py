@@ -128,6 +128,37 @@ def ob_linear_ln(X: torch.Tensor, W_packed: torch.Tensor, a: torch.Tensor, b: to
     return out
 
 
+def ob_stack_workspace_size() -> int:
+    return int(_lib.lib().ob_stack_workspace_size())
+
+
+def ob_linear_stack(layers, M: int, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Run a list of OneBit layers (M <= 16 tokens) in one persistent launch.
+
+    layers: sequence of (X, W_packed, a, b, Y, after_previous); X bf16 [M, K], W_packed int32
+    [N, K/32], a fp32 [N], b fp32 [K] or None, Y bf16/fp32 [M, N] (written), after_previous:
+    True if X is an output of an earlier layer of the list.
+    """
+    arr = (_lib.ObLayer * max(1, len(layers)))()
+    dev = None
+    for i, (X, P, a, b, Y, after) in enumerate(layers):
+        K = X.shape[1]
+        N = P.shape[0]
+        _need(X, "X", torch.bfloat16, (M, K))
+        _need(P, "W_packed", torch.int32, (N, K // 32))
+        _need(a, "a", torch.float32, (N,))
+        if b is not None:
+            _need(b, "b", torch.float32, (K,))
+        _need(Y, "Y", Y.dtype, (M, N))
+        arr[i] = _lib.ObLayer(_ptr(X), _ptr(P), _ptr(a), _ptr(b), _ptr(Y), K, N, _out_code(Y.dtype),
+                              1 if after else 0)
+        dev = X.device
+    if workspace is None:
+        workspace = torch.zeros(ob_stack_workspace_size(), dtype=torch.uint8, device=dev or "cuda")
+    st = _lib.lib().ob_linear_stack(arr, len(layers), M, _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check("ob_linear_stack", st)
+
+
 def dbf_workspace_size(M: int, r: int) -> int:
     return int(_lib.lib().dbf_workspace_size(M, r))
 

@@ -182,6 +182,49 @@ OB_API ob_status ob_linear_ln(const void* X, int64_t M, int64_t K,
                        const float* a, const float* b,
                        void* Z, int z_dtype, float eps, int path, void* stream);
 
+/*
+ * One layer of ob_linear_stack: Y = [(X ⊙ b^T) · W_sign^T] ⊙ a^T as in ob_linear.
+ *   X, W_packed, a, Y   device pointers as in ob_linear (X bf16 M x K, Y M x N).
+ *   b                   device fp32 [K], or NULL for no input scale.
+ *   K, N                K % 32 == 0, K >= 32, N >= 1.
+ *   y_dtype             ob_out_dtype of Y.
+ *   after_previous      nonzero if X is (or overlaps) the output of an earlier layer of
+ *                       the list: every earlier layer finishes before this one starts.
+ *                       Ignored for the first layer.
+ */
+typedef struct ob_layer {
+  const void* X;
+  const uint32_t* W_packed;
+  const float* a;
+  const float* b;
+  void* Y;
+  int64_t K;
+  int64_t N;
+  int32_t y_dtype;
+  int32_t after_previous;
+} ob_layer;
+
+/* Bytes of device workspace ob_linear_stack needs (its grid-barrier counter). */
+OB_API size_t ob_stack_workspace_size(void);
+
+/*
+ * A list of OneBit layers at M <= 16 tokens (decode) in one persistent cooperative
+ * launch per 384 layers, instead of one launch per layer: a decoder's layers read
+ * one another's outputs, and per-layer launches pay a launch and a drain for each.
+ * The layers between two after_previous flags run back to back; a flagged layer
+ * waits at a grid-wide barrier (bounded: a wait that runs out records
+ * OB_ERR_DEVICE_TIMEOUT for ob_last_device_error and the launch ends).  The pages
+ * have no counterpart: this is how their layer is applied layer after layer.
+ *   layers     HOST array of n_layers descriptors (read during the call only).
+ *   M          tokens, 0 <= M <= 16 (OB_ERR_SHAPE above).
+ *   workspace  device, at least ob_stack_workspace_size() bytes, not shared with a
+ *              concurrently running ob_linear_stack.
+ * Weights and scales must not be outputs of layers of the same list.  Validation of
+ * every descriptor happens before anything is launched.  Asynchronous.
+ */
+OB_API ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M,
+                          void* workspace, size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace dbf_linear needs (holds the M x r intermediate). */
 OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
 

@@ -1,0 +1,197 @@
+"""GPU parity of ob_linear_stack (a list of OneBit layers in one persistent launch).
+
+Every layer is checked against the fp64 oracle on the bf16 input it actually
+received (its X, possibly an earlier layer's Y), with the GEMM tolerances.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from binary_weight_gemm_b200 import synth
+from helpers import assert_gemm_close, oracle_svid
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ops():
+    from binary_weight_gemm_b200 import build
+    build.build()
+    from binary_weight_gemm_b200 import ops as _ops
+    torch.cuda.init()
+    return _ops
+
+
+def _cuda(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _x(xb):
+    return _cuda(xb.view(np.int16)).view(torch.bfloat16)
+
+
+def _np(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _layer(seed, N, K, scale_in=True):
+    W = synth.weights(seed, N, K)
+    a, b, _ = oracle.svid_rank1(W)
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    if not scale_in:
+        b = np.ones(K, dtype=np.float32)
+    return W, a, b
+
+
+def _check(layers_host, layer_io, what):
+    """layers_host: (W, a, b) per layer; layer_io: (X tensor, Y tensor) per layer after the run."""
+    for i, ((W, a, b), (X, Y)) in enumerate(zip(layers_host, layer_io)):
+        ref = oracle.onebit_linear(_np(X), oracle.sign_pm1(W), a, b)
+        assert_gemm_close(Y, ref, what=f"{what} layer {i}")
+
+
+@pytest.mark.parametrize("M", [1, 4, 9, 16])
+def test_stack_chain(ops, M):
+    K = 512
+    host = [_layer(200 + i, K, K) for i in range(8)]
+    X0 = _x(synth.activations(200, M, K)[0])
+    Ys = [torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for _ in host]
+    spec, x = [], X0
+    for i, ((W, a, b), Y) in enumerate(zip(host, Ys)):
+        spec.append((x, ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b), Y, i > 0))
+        x = Y
+    ops.ob_linear_stack(spec, M)
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    _check(host, [(s[0], s[4]) for s in spec], f"chain M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_stack_groups_ragged(ops, M):
+    # Group 1 (independent, all read X0): A 96->224, B 96->130 (fp32 out), C 96->64 without input
+    # scale.  Group 2 (after a barrier): D reads A (224->200), E reads A too (224->128, vector path).
+    X0 = _x(synth.activations(210, M, 96)[0])
+    shapes = [("A", 224, 96), ("B", 130, 96), ("C", 64, 96), ("D", 200, 224), ("E", 128, 224)]
+    host = {n: _layer(210 + i, N, K, scale_in=(n != "C")) for i, (n, N, K) in enumerate(shapes)}
+    out = {"A": torch.empty((M, 224), dtype=torch.bfloat16, device="cuda"),
+           "B": torch.empty((M, 130), dtype=torch.float32, device="cuda"),
+           "C": torch.empty((M, 64), dtype=torch.bfloat16, device="cuda"),
+           "D": torch.empty((M, 200), dtype=torch.bfloat16, device="cuda"),
+           "E": torch.empty((M, 128), dtype=torch.bfloat16, device="cuda")}
+    src = {"A": X0, "B": X0, "C": X0, "D": out["A"], "E": out["A"]}
+    spec = []
+    for n, N, K in shapes:
+        W, a, b = host[n]
+        spec.append((src[n], ops.ob_pack_signs(_cuda(W)), _cuda(a), None if n == "C" else _cuda(b), out[n],
+                     n == "D"))
+    ops.ob_linear_stack(spec, M)
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    _check([host[n] for n, _, _ in shapes], [(src[n], out[n]) for n, _, _ in shapes], f"groups M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_stack_dbf(ops, M):
+    # DBF as two layers: T = ((X ⊙ b) S_B^T) ⊙ m, then Y = (T S_A^T) ⊙ a (no input scale).
+    f = synth.dbf_factors(220, 1024, 512, 768)
+    xb, x = synth.activations(220, M, 768)
+    X = _x(xb)
+    T = torch.empty((M, 512), dtype=torch.bfloat16, device="cuda")
+    Y = torch.empty((M, 1024), dtype=torch.bfloat16, device="cuda")
+    SB = ops.ob_pack_signs(_cuda(f["S_B"].astype(np.float32)))
+    SA = ops.ob_pack_signs(_cuda(f["S_A"].astype(np.float32)))
+    ops.ob_linear_stack([(X, SB, _cuda(f["m"]), _cuda(f["b"]), T, False),
+                         (T, SA, _cuda(f["a"]), None, Y, True)], M)
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    assert_gemm_close(Y, oracle.dbf_linear(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"]), what=f"dbf stack M={M}")
+
+
+def test_stack_longer_than_one_launch(ops):
+    # 400 chained 64 x 64 layers: more than one launch's worth of descriptors.
+    M, K, L = 3, 64, 400
+    host = [_layer(1000 + i, K, K) for i in range(L)]
+    X0 = _x(synth.activations(230, M, K)[0])
+    Ys = [torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for _ in range(L)]
+    spec, x = [], X0
+    for i, ((W, a, b), Y) in enumerate(zip(host, Ys)):
+        spec.append((x, ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b), Y, i > 0))
+        x = Y
+    ops.ob_linear_stack(spec, M)
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    for i in (0, 1, 382, 383, 384, 385, L - 1):
+        W, a, b = host[i]
+        assert_gemm_close(Ys[i], oracle.onebit_linear(_np(spec[i][0]), oracle.sign_pm1(W), a, b),
+                          what=f"long stack layer {i}")
+
+
+def test_stack_in_cuda_graph(ops):
+    M, K = 4, 512
+    host = [_layer(240 + i, K, K) for i in range(4)]
+    X0 = _x(synth.activations(240, M, K)[0])
+    Ys = [torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for _ in host]
+    ws = torch.zeros(ops.ob_stack_workspace_size(), dtype=torch.uint8, device="cuda")
+    spec, x = [], X0
+    for i, ((W, a, b), Y) in enumerate(zip(host, Ys)):
+        spec.append((x, ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b), Y, i > 0))
+        x = Y
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ops.ob_linear_stack(spec, M, workspace=ws, stream=s)
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            ops.ob_linear_stack(spec, M, workspace=ws, stream=s)
+    for Y in Ys:
+        Y.zero_()
+    torch.cuda.synchronize()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    _check(host, [(sp[0], sp[4]) for sp in spec], "graph stack")
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_stack_7b_block(ops, M):
+    # One 7B-shaped block: q, k, v, o (4096 -> 4096), gate, up (4096 -> 11008), down (11008 -> 4096).
+    Wq, aq, bq, _ = oracle_svid(1, 4096, 4096)
+    Wg, ag, bg, _ = oracle_svid(5, 11008, 4096)
+    Wd, ad, bd, _ = oracle_svid(6, 4096, 11008)
+    X0 = _x(synth.activations(250, M, 4096, outliers=True)[0])
+    Pq, Pg, Pd = (ops.ob_pack_signs(_cuda(W)) for W in (Wq, Wg, Wd))
+    buf = {n: torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+           for n, N in (("q", 4096), ("k", 4096), ("v", 4096), ("o", 4096), ("gate", 11008), ("up", 11008),
+                        ("down", 4096))}
+    P = {"q": (Pq, aq, bq, Wq), "k": (Pq, aq, bq, Wq), "v": (Pq, aq, bq, Wq), "o": (Pq, aq, bq, Wq),
+         "gate": (Pg, ag, bg, Wg), "up": (Pg, ag, bg, Wg), "down": (Pd, ad, bd, Wd)}
+    src = {"q": X0, "k": X0, "v": X0, "o": buf["q"], "gate": buf["o"], "up": buf["o"], "down": buf["gate"]}
+    after = {"o": True, "gate": True, "down": True}
+    order = ["q", "k", "v", "o", "gate", "up", "down"]
+    spec = [(src[n], P[n][0], _cuda(P[n][1]), _cuda(P[n][2]), buf[n], after.get(n, False)) for n in order]
+    ops.ob_linear_stack(spec, M)
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    for n in order:
+        W, a, b = P[n][3], P[n][1], P[n][2]
+        assert_gemm_close(buf[n], oracle.onebit_linear(_np(src[n]), oracle.sign_pm1(W), a, b),
+                          what=f"7b block {n} M={M}")
+
+
+def test_stack_argument_errors(ops):
+    from binary_weight_gemm_b200._lib import ObError
+    K = 64
+    W, a, b = _layer(260, 32, K)
+    P = ops.ob_pack_signs(_cuda(W))
+    X = torch.zeros((17, K), dtype=torch.bfloat16, device="cuda")
+    Y = torch.empty((17, 32), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ObError):  # M > 16
+        ops.ob_linear_stack([(X, P, _cuda(a), _cuda(b), Y, False)], 17)
+    X4, Y4 = X[:4].contiguous(), Y[:4].contiguous()
+    with pytest.raises(ObError):  # workspace too small
+        ops.ob_linear_stack([(X4, P, _cuda(a), _cuda(b), Y4, False)], 4,
+                            workspace=torch.zeros(16, dtype=torch.uint8, device="cuda"))
+    ops.ob_linear_stack([], 4)  # empty list: nothing to do
+    assert ops.ob_last_device_error() == 0
