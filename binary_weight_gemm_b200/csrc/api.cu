@@ -254,9 +254,23 @@ ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M, void*
   return status_of(launch_sign_stack(host.data(), n_layers, M, static_cast<unsigned*>(workspace), c));
 }
 
+// Bytes of the bf16 intermediate T: the smallest workspace dbf_linear accepts.
+size_t dbf_t_bytes(int64_t M, int64_t r) { return align256((size_t)M * (size_t)r * 2); }
+
+// K slices of DBF's first product (T = ... S_B^T, M x r) when it runs on the tcgen05 GEMM.
+int dbf_split_k(int64_t M, int64_t r, int num_sms) {
+  return M > decode_max_m() ? tc_split_k(M, r, num_sms) : 1;
+}
+
+int sms_for_sizing() {
+  DeviceInfo d;
+  return current_device(&d) == OB_OK && d.num_sms > 0 ? d.num_sms : 148;  // B200 when no device
+}
+
 size_t dbf_workspace_size(int64_t M, int64_t r) {
   if (M < 0 || r < 0) return 0;
-  return align256((size_t)M * (size_t)r * 2);
+  const int ks = dbf_split_k(M, r, sms_for_sizing());
+  return dbf_t_bytes(M, r) + (ks > 1 ? align256((size_t)ks * (size_t)M * (size_t)r * 4) : 0);
 }
 
 ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_packed, int64_t r, const float* m,
@@ -274,7 +288,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
                      misaligned(b)))
     return OB_ERR_ALIGN;
   if (!empty_sum) {
-    if (!workspace || ws_bytes < dbf_workspace_size(M, r)) return OB_ERR_WORKSPACE;
+    if (!workspace || ws_bytes < dbf_t_bytes(M, r)) return OB_ERR_WORKSPACE;
     if (misaligned(workspace)) return OB_ERR_ALIGN;
   }
   LaunchCtx c;
@@ -284,9 +298,27 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   // T = ((X ⊙ b^T) S_B^T) ⊙ m^T, rounded once to bf16, then Y = (T S_A^T) ⊙ a^T.
   uint16_t* T = static_cast<uint16_t*>(workspace);
   SignGemmArgs g1{static_cast<const uint16_t*>(X), M, K, SB_packed, r, b, m, T, r, OB_OUT_BF16};
-  st = run_sign_gemm(g1, path, c);
+  // Few output tiles (small M x r): split the first product over K into fp32 partial
+  // sums after T in the workspace, when the workspace holds them.
+  const bool tc1 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > decode_max_m() && K <= sign_gemm_tc_max_k());
+  const int ks = tc1 ? dbf_split_k(M, r, c.num_sms) : 1;
+  const size_t part_off = dbf_t_bytes(M, r);
+  if (ks > 1 && path != OB_PATH_TC_DECODE && ws_bytes >= part_off + (size_t)ks * (size_t)M * (size_t)r * 4) {
+    g1.l2_prefetch = 0;
+    st = status_of(launch_sign_gemm_tc_splitk(
+        g1, ks, reinterpret_cast<float*>(static_cast<char*>(workspace) + part_off), c));
+  } else {
+    st = run_sign_gemm(g1, path, c);
+  }
   if (st != OB_OK) return st;
   SignGemmArgs g2{T, M, r, SA_packed, N, nullptr, a, Y, N, y_dtype};
+  // The second product splits the same way when the region after T also holds its
+  // partial sums (the first product's are consumed before it runs).
+  const bool tc2 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > decode_max_m() && r <= sign_gemm_tc_max_k());
+  const int ks2 = tc2 && M > decode_max_m() ? tc_split_k(M, N, c.num_sms) : 1;
+  if (ks2 > 1 && ws_bytes >= part_off + (size_t)ks2 * (size_t)M * (size_t)N * 4)
+    return status_of(launch_sign_gemm_tc_splitk(
+        g2, ks2, reinterpret_cast<float*>(static_cast<char*>(workspace) + part_off), c));
   return run_sign_gemm(g2, path, c);
 }
 

@@ -47,6 +47,7 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(kRows, kTok);
 // K = 16384, three up to K = 32768.
 constexpr int64_t kMaxK4 = 16384;
 constexpr int64_t kMaxK = 32768;
+constexpr int kOutDirect = 0, kOutTmaStore = 1, kOutSplit = 2;  // epilogue modes
 
 struct __align__(128) TcShared {  // 128-byte size keeps the bf16x2 table after it 16-byte aligned
   uint64_t full[kMaxStages];   // X tile landed (TMA transaction bytes) and all four A warps stored
@@ -81,7 +82,8 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, unsign
 template <int kStages>
 __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                     const __grid_constant__ CUtensorMap tmap_y,
-                                                                    SignGemmArgs g, int tma_store, unsigned* err) {
+                                                                    SignGemmArgs g, int out_mode, int ksplit,
+                                                                    float* part, unsigned* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // [ring: kStages x 32 KB][output tile 64 KB][TcShared][iscale pairs]
   uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -95,6 +97,15 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
   const int64_t m_blocks = (g.M + kTok - 1) / kTok;
   const int64_t n_blocks = (g.R + kRows - 1) / kRows;
   const int64_t tiles = m_blocks * n_blocks;
+  // Work unit u = (tile u / ksplit, k slice u % ksplit).  Slices are whole groups of
+  // four stages (8 packed words), so every slice starts 16-byte aligned.
+  const int ngroups_k = (nkb + 3) / 4;
+  const int64_t units = tiles * ksplit;
+  auto unit_k = [&](int64_t u, int& kb0, int& kb1) {
+    const int ks = (int)(u % ksplit);
+    kb0 = 4 * (int)((int64_t)ks * ngroups_k / ksplit);
+    kb1 = std::min(nkb, 4 * (int)((int64_t)(ks + 1) * ngroups_k / ksplit));
+  };
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -134,12 +145,15 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     const bool vec = (Wd & 3) == 0;
     int64_t gstage = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+    for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      const int64_t tile = u / ksplit;
+      int kb0, kb1;
+      unit_k(u, kb0, kb1);
       const int64_t n = (tile % n_blocks) * kRows + tid;
       const bool row_ok = n < g.R;
       const uint32_t* srow = g.S + (row_ok ? n : 0) * Wd;
       auto load_group = [&](int64_t grp, uint32_t (&wv)[8]) {
-        const int64_t w0 = grp * 8;
+        const int64_t w0 = 2 * (int64_t)kb0 + grp * 8;
         if (vec) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -154,13 +168,13 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
       };
       uint32_t cur[8], nxt[8];
       load_group(0, cur);
-      const int ngroups = (nkb + 3) / 4;
+      const int ngroups = (kb1 - kb0 + 3) / 4;
       for (int grp = 0; grp < ngroups && ok; ++grp) {
         load_group(grp + 1, nxt);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int kb = grp * 4 + i;
-          if (kb >= nkb) break;
+          const int kb = kb0 + grp * 4 + i;
+          if (kb >= kb1) break;
           const uint32_t w0 = cur[2 * i], w1 = cur[2 * i + 1];
           const int s = (int)(gstage % kStages);
           if (gstage >= kStages) {
@@ -207,13 +221,42 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int c0 = half * (kTok / 64), c1 = c0 + kTok / 64;
     int64_t it = 0;
-    if (tma_store) {
+    if (out_mode == kOutSplit) {
+      // Split K: this unit's fp32 partial sums, unscaled, to part[k slice][m][n];
+      // a second kernel sums the slices and applies the output scale.
+      for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+        if (!wait_warp(&sh->dfull, (uint32_t)it & 1u, err, abort_flag, lane)) break;
+        tc_fence_after();
+        const int64_t tile = u / ksplit, ks = u % ksplit;
+        const int64_t m0 = (tile / n_blocks) * kTok;
+        const int64_t nr = (tile % n_blocks) * kRows + q * 32 + lane;
+        float* dst = part + (ks * g.M) * g.R + nr;
+#pragma unroll 1
+        for (int c = c0; c < c1; ++c) {
+          uint32_t d[32];
+          tmem_ld_x32(lane_base + 32u * c, d);
+          tmem_wait_ld();
+          if (c == c1 - 1) {  // this warp's last read of the accumulator
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh->dempty);
+          }
+          if (nr < g.R) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int64_t m = m0 + 32 * c + i;
+              if (m < g.M) dst[m * g.R] = __uint_as_float(d[i]);
+            }
+          }
+        }
+      }
+    } else if (out_mode == kOutTmaStore) {
       // bf16 Y: the tile is staged in shared memory as [token][row], Y's own
       // layout, and written by one TMA store that clips the ragged edges.  The
       // accumulator is released right after its last tcgen05.ld, so the next
       // tile's MMAs overlap the conversion and the store.
       uint16_t* col = reinterpret_cast<uint16_t*>(out_tile) + q * 32 + lane;
-      for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+      for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {  // ksplit == 1
         if (!wait_warp(&sh->dfull, (uint32_t)it & 1u, err, abort_flag, lane)) break;
         tc_fence_after();
         if (it > 0 && !wait_warp(&sh->stg_free, (uint32_t)(it - 1) & 1u, err, abort_flag, lane)) break;
@@ -256,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
       float* scr = reinterpret_cast<float*>(out_tile) + (warp - 4) * (32 * 33);
       const bool f32 = g.y_dtype == OB_OUT_F32;
       const bool vec_ok = (g.ldy % (f32 ? 4 : 8)) == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0;
-      for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+      for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {  // ksplit == 1
         if (!wait_warp(&sh->dfull, (uint32_t)it & 1u, err, abort_flag, lane)) break;
         tc_fence_after();
         const int64_t m0 = (tile / n_blocks) * kTok;
@@ -323,9 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
       prefetch_tmap(&tmap_x);
         int64_t gstage = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        const int32_t m0 = (int32_t)((tile / n_blocks) * kTok);
-        for (int kb = 0; kb < nkb; ++kb, ++gstage) {
+      for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int32_t m0 = (int32_t)((u / ksplit / n_blocks) * kTok);
+        int kb0, kb1;
+        unit_k(u, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++gstage) {
           const int s = (int)(gstage % kStages);
           if (gstage >= kStages) {
             ok = mbar_wait(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag);
@@ -348,13 +393,15 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
       uint32_t s = 0, phase = 0;
       int64_t it = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++it) {
+      for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
         if (it > 0) {
           ok = mbar_wait(&sh->dempty, (uint32_t)(it - 1) & 1u, err, abort_flag);
           if (!ok) break;
           tc_fence_after();
         }
-        for (int kb = 0; kb < nkb; ++kb) {
+        int kb0, kb1;
+        unit_k(u, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           // One barrier per stage for both operands: a second wait costs the issuing
           // thread about a hundred cycles per stage.
           ok = mbar_wait(&sh->full[s], phase, err, abort_flag);
@@ -366,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
           const uint64_t so = (uint64_t)(s * (kXStageBytes >> 4));
           const uint64_t b0 = d0 + so, b1 = d1 + so, b2 = d2 + so, b3 = d3 + so;
           const uint32_t aa = tmem + 256u + 32u * s;
-          mma_bf16_ts(tmem, aa, b0, kIdesc, kb > 0 ? 1u : 0u);
+          mma_bf16_ts(tmem, aa, b0, kIdesc, kb > kb0 ? 1u : 0u);
           mma_bf16_ts(tmem, aa + 8u, b1, kIdesc, 1u);
           if ((int64_t)(kb + 1) * kBK <= K) {  // a trailing half stage holds 32 k
             mma_bf16_ts(tmem, aa + 16u, b2, kIdesc, 1u);
@@ -415,7 +462,39 @@ EncodeTiledFn get_encode_fn() {
 
 int64_t sign_gemm_tc_max_k() { return kMaxK; }
 
-cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
+int tc_split_k(int64_t M, int64_t R, int num_sms) {
+  const int64_t tiles = ((M + kTok - 1) / kTok) * ((R + kRows - 1) / kRows);
+  if (tiles == 0 || tiles * 2 > num_sms) return 1;
+  return (int)std::min<int64_t>(8, num_sms / tiles);
+}
+
+namespace {
+
+// Y[m, n] = oscale[n] * sum over k slices of part[slice][m][n]; 4 consecutive n per item.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* part, int ksplit, int64_t M, int64_t R,
+                                                            const float* oscale, void* Y, int64_t ldy, int y_dtype) {
+  pdl_wait();  // the partial sums come from the previous grid
+  pdl_launch_dependents();
+  const int64_t r4 = R / 4, items = M * r4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < items; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = i / r4, n = (i - m * r4) * 4;
+    float4 acc = __ldcg(reinterpret_cast<const float4*>(part + m * R + n));
+    for (int ks = 1; ks < ksplit; ++ks) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(part + ((int64_t)ks * M + m) * R + n));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const float4 sc = __ldg(reinterpret_cast<const float4*>(oscale + n));
+    acc.x *= sc.x; acc.y *= sc.y; acc.z *= sc.z; acc.w *= sc.w;
+    if (y_dtype == OB_OUT_F32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(Y) + m * ldy + n) = acc;
+    } else {
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(Y) + m * ldy + n) =
+          make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    }
+  }
+}
+
+cudaError_t launch_tc_impl(const SignGemmArgs& g, int ksplit, float* part, const LaunchCtx& c) {
   if (g.M == 0 || g.R == 0 || g.K == 0) return cudaSuccess;
   if (g.K > kMaxK) return cudaErrorInvalidValue;
   EncodeTiledFn encode = get_encode_fn();
@@ -436,7 +515,7 @@ cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
   }
   // bf16 Y whose rows start on 16-byte boundaries is written by TMA stores.
   int tma_store = 0;
-  if (g.y_dtype == OB_OUT_BF16 && g.ldy % 8 == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0) {
+  if (ksplit == 1 && g.y_dtype == OB_OUT_BF16 && g.ldy % 8 == 0 && (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0) {
     const cuuint64_t dims[2] = {(cuuint64_t)g.R, (cuuint64_t)g.M};
     const cuuint64_t strides[1] = {(cuuint64_t)g.ldy * 2};
     const cuuint32_t box[2] = {(cuuint32_t)kRows, (cuuint32_t)kTok};
@@ -448,7 +527,8 @@ cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
   }
 
   const int64_t tiles = ((g.M + kTok - 1) / kTok) * ((g.R + kRows - 1) / kRows);
-  const int grid = (int)std::min<int64_t>(tiles, c.num_sms);
+  const int grid = (int)std::min<int64_t>(tiles * ksplit, c.num_sms);
+  const int out_mode = ksplit > 1 ? kOutSplit : (tma_store ? kOutTmaStore : kOutDirect);
   const int stages = g.K <= kMaxK4 ? 4 : 3;
   const size_t smem = 1024 + (size_t)stages * kXStageBytes + kOutTileBytes + sizeof(TcShared) +
                       sizeof(uint32_t) * ((((g.K + 1) / 2) + 3) & ~int64_t(3));
@@ -470,7 +550,36 @@ cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) {
   auto kern = stages == 4 ? sign_gemm_tc_kernel<4> : sign_gemm_tc_kernel<3>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = cudaLaunchKernelEx(&cfg, kern, tmap_x, tmap_y, g, tma_store, c.err);
+  e = cudaLaunchKernelEx(&cfg, kern, tmap_x, tmap_y, g, out_mode, ksplit, part, c.err);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) { return launch_tc_impl(g, 1, nullptr, c); }
+
+cudaError_t launch_sign_gemm_tc_splitk(const SignGemmArgs& g, int ksplit, float* part, const LaunchCtx& c) {
+  if (g.M == 0 || g.R == 0 || g.K == 0) return cudaSuccess;
+  // K slices are whole 4-stage groups, and at least 16 stages (1024 k) long: shorter
+  // slices cost more in the extra partial-sum pass than they gain (measured on B200).
+  const int64_t nkb = (g.K + kBK - 1) / kBK;
+  ksplit = (int)std::min<int64_t>(ksplit, std::min<int64_t>((nkb + 3) / 4, nkb / 16));
+  if (ksplit <= 1 || g.R % 4 != 0 || g.ldy % 4 != 0) return launch_tc_impl(g, 1, nullptr, c);
+  cudaError_t e = launch_tc_impl(g, ksplit, part, c);
+  if (e != cudaSuccess) return e;
+  const int64_t items = g.M * (g.R / 4);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::min<int64_t>((items + 255) / 256, (int64_t)c.num_sms * 8), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = c.pdl ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, static_cast<const float*>(part), ksplit, g.M, g.R, g.oscale,
+                         g.Y, g.ldy, g.y_dtype);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -41,6 +41,14 @@ cudaError_t launch_sign_gemm_mma_decode(const SignGemmArgs& g, const LaunchCtx& 
 cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c);
 // Largest K the tcgen05 GEMM takes (its input-scale pairs live in shared memory).
 int64_t sign_gemm_tc_max_k();
+// K slices for the tcgen05 GEMM of an M x R output: more than one when the output has
+// fewer 128 x 256 tiles than half the SMs (at most 8).
+int tc_split_k(int64_t M, int64_t R, int num_sms);
+// The tcgen05 GEMM split over K: fp32 partial sums of each slice into part
+// (ksplit x M x R floats), then a reduction that applies oscale and writes Y.
+// Slices hold at least 1024 k; falls back to the unsplit kernel when K is too short for
+// two slices or R, ldy are not multiples of 4.
+cudaError_t launch_sign_gemm_tc_splitk(const SignGemmArgs& g, int ksplit, float* part, const LaunchCtx& c);
 
 // SVID power iteration pieces (see svid.cu).
 size_t svid_workspace_bytes(int64_t N, int64_t K);

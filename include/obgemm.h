@@ -225,7 +225,14 @@ OB_API size_t ob_stack_workspace_size(void);
 OB_API ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M,
                           void* workspace, size_t ws_bytes, void* stream);
 
-/* Bytes of device workspace dbf_linear needs (holds the M x r intermediate). */
+/*
+ * Bytes of device workspace dbf_linear uses: the M x r bf16 intermediate T and, when
+ * the first product runs on the tcgen05 GEMM with fewer output tiles than half the
+ * SMs of the current device (e.g. M = 512, r = 2048), fp32 partial sums for splitting
+ * it over K (up to 8 x M x r x 4 bytes).  dbf_linear accepts any workspace of at least
+ * the intermediate's size (M x r x 2 rounded up to 256 bytes); a smaller one than
+ * this function returns runs the first product without the split.
+ */
 OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
 
 /*
