@@ -104,7 +104,8 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
   auto unit_k = [&](int64_t u, int& kb0, int& kb1) {
     const int ks = (int)(u % ksplit);
     kb0 = 4 * (int)((int64_t)ks * ngroups_k / ksplit);
-    kb1 = std::min(nkb, 4 * (int)((int64_t)(ks + 1) * ngroups_k / ksplit));
+    const int end = 4 * (int)((int64_t)(ks + 1) * ngroups_k / ksplit);
+    kb1 = end < nkb ? end : nkb;
   };
 
   if (tid == 0) {
