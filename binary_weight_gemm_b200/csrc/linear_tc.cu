@@ -146,6 +146,18 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
     const bool vec = (Wd & 3) == 0;
     int64_t gstage = 0;
     bool ok = true;
+    // A stage's tcgen05.st is waited for only after the next stage's values are
+    // computed: store latency overlaps the expansion arithmetic.
+    int pending = -1;
+    auto flush_pending = [&]() {
+      if (pending >= 0) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->full[pending]);
+        pending = -1;
+      }
+    };
     for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const int64_t tile = u / ksplit;
       int kb0, kb1;
@@ -177,12 +189,6 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
           const int kb = kb0 + grp * 4 + i;
           if (kb >= kb1) break;
           const uint32_t w0 = cur[2 * i], w1 = cur[2 * i + 1];
-          const int s = (int)(gstage % kStages);
-          if (gstage >= kStages) {
-            ok = wait_warp(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag, lane);
-            if (!ok) break;
-            tc_fence_after();
-          }
           const uint4* bp = reinterpret_cast<const uint4*>(bpair + (int64_t)kb * (kBK / 2));
           const bool full_stage = (int64_t)(kb + 1) * kBK <= K;
           // Column c of the stage holds k = 2c, 2c+1.  After unzip_bits, bit j of a
@@ -202,17 +208,25 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc_kernel(const __grid_
               v[c] = ((u << (15 - (c & 15))) & 0x80008000u) ^ bb[e];
             }
           }
+          // The previous stage's store has had this stage's arithmetic to land: only
+          // now wait for it and release that stage to the MMA.
+          flush_pending();
+          const int s = (int)(gstage % kStages);
+          if (gstage >= kStages) {
+            ok = wait_warp(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag, lane);
+            if (!ok) break;
+            tc_fence_after();
+          }
           tmem_st_x32(lane_base + 256u + 32u * s, v);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->full[s]);
+          pending = s;
           ++gstage;
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
       }
+      flush_pending();  // the tile's last stage, before the next tile's sign loads
     }
+    flush_pending();
   } else if (warp < 12) {
     // ------------------------------------------------ epilogue
     // Two warps per TMEM lane quadrant; a thread holds one weight row of the
