@@ -107,7 +107,12 @@ ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) 
     case OB_PATH_SIMT: e = launch_sign_gemm_simt(g, c); break;
     case OB_PATH_TC_DECODE: e = launch_sign_gemm_tc_decode(g, c); break;
     case OB_PATH_MMA_DECODE: e = launch_sign_gemm_mma_decode(g, c); break;
-    case OB_PATH_TC: e = launch_sign_gemm_tc(g, c); break;
+    case OB_PATH_TC:
+      // The CTA-pair kernel is opt-in (OB_TC2=1): on B200 it measured slower than the
+      // one-CTA kernel at the prefill workload (773 vs 1189 TFLOP/s).
+      e = (env_flag("OB_TC2", false) && sign_gemm_tc2_supported(g)) ? launch_sign_gemm_tc2(g, c)
+                                                                    : launch_sign_gemm_tc(g, c);
+      break;
     default: return OB_ERR_UNSUPPORTED;
   }
   return status_of(e);

@@ -477,6 +477,8 @@ EncodeTiledFn get_encode_fn() {
 
 int64_t sign_gemm_tc_max_k() { return kMaxK; }
 
+void* tensor_map_encode_tiled_fn() { return reinterpret_cast<void*>(get_encode_fn()); }
+
 int tc_split_k(int64_t M, int64_t R, int num_sms) {
   const int64_t tiles = ((M + kTok - 1) / kTok) * ((R + kRows - 1) / kRows);
   if (tiles == 0 || tiles * 2 > num_sms) return 1;

@@ -39,6 +39,14 @@ cudaError_t launch_sign_gemm_simt(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_tc_decode(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_mma_decode(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c);
+// cuTensorMapEncodeTiled from the driver (null if unavailable).
+void* tensor_map_encode_tiled_fn();
+
+// The CTA-pair tcgen05 GEMM (linear_tc2.cu): bf16 Y with 16-byte-aligned rows,
+// K <= 16384, M >= 512, R >= 256.
+bool sign_gemm_tc2_supported(const SignGemmArgs& g);
+cudaError_t launch_sign_gemm_tc2(const SignGemmArgs& g, const LaunchCtx& c);
+
 // Largest K the tcgen05 GEMM takes (its input-scale pairs live in shared memory).
 int64_t sign_gemm_tc_max_k();
 // K slices for the tcgen05 GEMM of an M x R output: more than one when the output has
