@@ -44,6 +44,9 @@ constexpr uint32_t kOutTileBytes = kTok * kRowsCta * 2;   // 64 KB bf16 output t
 constexpr int kTmemCols = 512;                            // D [0,256), A slots 256 + 64*s
 constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kRowsCta, kTok);
 constexpr int64_t kMaxK = 16384;
+// Warp roles: 0-7 expand signs (two per TMEM lane quadrant, each half of a stage's
+// 64 columns), 8-11 epilogue (one per quadrant), 12 TMA, 13 MMA (rank 0) + TMEM.
+constexpr int kAWarps = 8, kEpiWarps = 4, kEpiWarp0 = 8, kTmaWarp = 12, kMmaWarp = 13;
 
 struct __align__(128) Tc2Shared {
   uint64_t full[kStages];  // rank 0: both CTAs' TMA bytes + 8 expansion warps + rank 0's TMA arrival
@@ -94,12 +97,12 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sh->full[s], 9);
+      mbar_init(&sh->full[s], 1 + 2 * kAWarps);  // rank 0's TMA arrival + both CTAs' A warps
       mbar_init(&sh->empty[s], 1);
     }
     mbar_init(&sh->dfull, 1);
-    mbar_init(&sh->dempty, 16);
-    mbar_init(&sh->stg_full, 8);
+    mbar_init(&sh->dempty, 2 * kEpiWarps);
+    mbar_init(&sh->stg_full, kEpiWarps);
     mbar_init(&sh->stg_free, 1);
     sh->abort_flag = 0;
     fence_mbar_init();
@@ -110,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
     const float hi = g.iscale ? __ldg(g.iscale + 2 * i + 1) : 1.f;
     bpair[i] = pack_bf16x2(lo, hi);
   }
-  if (warp == 13) {
+  if (warp == kMmaWarp) {
     tmem_alloc_pair(&sh->tmem_base, kTmemCols);
     tmem_relinquish_pair();
   }
@@ -124,14 +127,17 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
   const uint32_t full0 = mapa_shared(&sh->full[0], 0);
   const uint32_t dempty0 = mapa_shared(&sh->dempty, 0);
 
-  if (warp < 4) {
+  if (warp < kAWarps) {
     // ------------------------------------------------ A producer: this CTA's 128 weight rows
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // Warp w: TMEM lane quadrant w % 4 (32 rows), column half w / 4 of each stage
+    // (32 columns = two packed words = 64 k).
+    const int aq = warp & 3, ahalf = warp >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)(aq * 32) << 16);
     const bool vec = (Wd & 3) == 0;
     int64_t gstage = 0;
     bool ok = true;
     for (int64_t tile = pair; tile < tiles && ok; tile += npairs) {
-      const int64_t n = (tile % n_blocks) * (2 * kRowsCta) + rank * kRowsCta + tid;
+      const int64_t n = (tile % n_blocks) * (2 * kRowsCta) + rank * kRowsCta + aq * 32 + lane;
       const bool row_ok = n < g.R;
       const uint32_t* srow = g.S + (row_ok ? n : 0) * Wd;
       // 8 words = two stages, fetched a group ahead.
@@ -169,9 +175,12 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
           const int64_t left = K - (int64_t)kb * kBK;
           const int valid = (int)(left < kBK ? left : kBK) / 2;
           const uint4* bp = reinterpret_cast<const uint4*>(bpair + (int64_t)kb * (kBK / 2));
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint32_t u0 = unzip_bits2(cur[4 * i + 2 * half]), u1 = unzip_bits2(cur[4 * i + 2 * half + 1]);
+          {
+            const int half = ahalf;
+            // Selects keep cur in registers (no runtime index into it).
+            const uint32_t wa = i ? (half ? cur[6] : cur[4]) : (half ? cur[2] : cur[0]);
+            const uint32_t wb = i ? (half ? cur[7] : cur[5]) : (half ? cur[3] : cur[1]);
+            const uint32_t u0 = unzip_bits2(wa), u1 = unzip_bits2(wb);
             uint32_t v[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -198,12 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
         for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
       }
     }
-  } else if (warp < 12) {
+  } else if (warp < kEpiWarp0 + kEpiWarps) {
     // ------------------------------------------------ epilogue: this CTA's 128 rows x 256 tokens
     const int q = warp & 3;
-    const int half = (warp - 4) >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    const int c0 = half * (kTok / 64), c1 = c0 + kTok / 64;
+    const int c0 = 0, c1 = kTok / 32;
     uint16_t* col = reinterpret_cast<uint16_t*>(out_tile) + q * 32 + lane;
     int64_t it = 0;
     for (int64_t tile = pair; tile < tiles; tile += npairs, ++it) {
@@ -231,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->stg_full);
-      if (warp == 4 && lane == 0) {
+      if (warp == kEpiWarp0 && lane == 0) {
         if (mbar_wait(&sh->stg_full, (uint32_t)it & 1u, err, abort_flag)) {
           tma_store_2d(&tmap_y, out_tile, (int32_t)n0, (int32_t)m0);
           bulk_commit_group();
@@ -241,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
       }
       __syncwarp();
     }
-    if (warp == 4 && lane == 0) bulk_wait_all();
-  } else if (warp == 12) {
+    if (warp == kEpiWarp0 && lane == 0) bulk_wait_all();
+  } else if (warp == kTmaWarp) {
     // ------------------------------------------------ TMA producer: this CTA's 128 tokens
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
@@ -306,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // no MMA, remote arrival or TMA of the pair is still outstanding
-  if (warp == 13) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, kTmemCols);
   }
