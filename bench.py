@@ -165,6 +165,16 @@ def load_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def prefill_kernel_name() -> str:
+    """The tcgen05 GEMM the prefill workload runs: the CTA-pair kernel unless OB_TC2=0."""
+    return "sign_gemm_tc_kernel" if os.environ.get("OB_TC2", "1")[:1] in ("0", "n", "N", "f", "F") \
+        else "sign_gemm_tc2_kernel"
+
+
+def prefill_kernel_source():
+    return ("linear_tc.cu",) if prefill_kernel_name() == "sign_gemm_tc_kernel" else ("linear_tc2.cu",)
+
+
 def ncu_traffic(kernel_file: str, key: str):
     """DRAM bytes per launch from a committed ncu summary, or None if the kernel changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -531,8 +541,8 @@ def run_prefill(args, world, rank, local):
             "roofline": {"bound": "tensor", "achieved": flops / t / 1e12, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": flops / t / 1e12 / peaks["bf16_tflops"],
                          "frac_sustained": flops / t / 1e12 / (peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]),
-                         "peak_source": peaks["source"], "kernel": "sign_gemm_tc_kernel",
-                         "traffic": ncu_traffic("linear_tc.cu", "prefill_2048x4096x11008")},
+                         "peak_source": peaks["source"], "kernel": prefill_kernel_name(),
+                         "traffic": ncu_traffic(*prefill_kernel_source(), "prefill_2048x4096x11008")},
             "e2e": {"value": world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N},
             "gpu_launches": args.steps, "clocks": clocks, "cpu_baseline": cpu,
@@ -715,13 +725,13 @@ def run_extra(ops, dev, stream, peaks):
     out["prefill_2048x4096x11008"] = {"us_per_call": t * 1e6, "tflops": fl / t / 1e12,
                                       "frac_bf16_burst": fl / t / 1e12 / peaks["bf16_tflops"],
                                       "frac_bf16_sustained": fl / t / 1e12 / (peaks["bf16_tflops_sustained"] or 1),
-                                      "kernel": "sign_gemm_tc_kernel"}
+                                      "kernel": prefill_kernel_name()}
     # The same prefill followed by LayerNorm over each token's outputs (ob_linear_ln).
     t_ln = _time_calls(lambda i: ops.ob_linear_ln(sets[i % 3][0], sets[i % 3][1], a, b, out=sets[i % 3][2],
                                                   stream=stream), stream, 30)
     out["prefill_ln_2048x4096x11008"] = {"us_per_call": t_ln * 1e6, "tflops": fl / t_ln / 1e12,
                                          "ln_us": (t_ln - t) * 1e6,
-                                         "kernels": "sign_gemm_tc_kernel + layernorm_rows_kernel"}
+                                         "kernels": prefill_kernel_name() + " + layernorm_rows_kernel"}
     del sets
     # OneBit decode 4096 x 4096 followed by LayerNorm, M = 1 and 16 (pool of weight sets > L2).
     W = torch.from_numpy(synth.weights(1, 4096, 4096)).to(dev)

@@ -85,7 +85,8 @@ typedef enum ob_path {
   OB_PATH_AUTO = 0,        /* M == 1: OB_PATH_SIMT; M <= 16 or K > 32768: OB_PATH_MMA_DECODE; else OB_PATH_TC */
   OB_PATH_SIMT = 1,        /* CUDA-core select/add mat-vec (any M; slow for M > 4) */
   OB_PATH_TC_DECODE = 2,   /* tcgen05, signs unpacked into tensor memory, M <= 16 per pass */
-  OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA); K <= 32768 */
+  OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA); K <= 32768; a
+                              2-CTA (cta_group::2) tile where bf16 Y, M >= 512, N >= 256, K <= 16384 */
   OB_PATH_MMA_DECODE = 4   /* warp-level MMA, signs unpacked in registers, M <= 16 per pass */
 } ob_path;
 

@@ -1,7 +1,8 @@
 """GPU parity of the CTA-pair tcgen05 GEMM (linear_tc2.cu) against the fp64 oracle.
 
-With OB_TC2=1, OB_PATH_TC with bf16 output, M >= 512 and N >= 256 runs the pair
-kernel; these shapes exercise its ragged tiles: N not a multiple of 256
+OB_PATH_TC (and AUTO above 16 tokens) with bf16 output, M >= 512 and N >= 256 runs
+the pair kernel (OB_TC2=0 selects the one-CTA kernel); these shapes exercise its
+ragged tiles: N not a multiple of 256
 (a pair whose second CTA has no valid rows), M not a multiple of 256, K with a
 partial 128-k stage.
 """
