@@ -94,3 +94,42 @@ def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_LIB", None)
     with pytest.raises(ImportError):
         _lib.lib()
+
+
+def test_layernorm_and_stack_argument_checks_without_gpu(lib):
+    from binary_weight_gemm_b200._lib import ObLayer
+    OK, NULL, SHAPE, ALIGN, WS, UNSUP = 0, 1, 2, 3, 6, 9
+    p = ctypes.c_void_p(4096)
+    bad = ctypes.c_void_p(4100)
+    # ob_linear_ln: eps is checked before anything else; then the ob_linear checks.
+    for eps in (-1.0, float("nan"), float("inf")):
+        assert lib.ob_linear_ln(p, 1, 64, p, 4, p, p, p, 0, eps, 0, None) == UNSUP
+    assert lib.ob_linear_ln(p, 1, 48, p, 4, p, p, p, 0, 1e-5, 0, None) == SHAPE
+    assert lib.ob_linear_ln(None, 0, 64, None, 8, None, None, None, 0, 1e-5, 0, None) == OK
+    assert lib.ob_linear_ln(p, 1, 64, p, 4, p, p, None, 0, 1e-5, 0, None) == NULL
+    # ob_linear_stack: every descriptor is validated before a launch.
+    assert lib.ob_stack_workspace_size() >= 8
+
+    def layers(*descs):
+        arr = (ObLayer * len(descs))()
+        for i, d in enumerate(descs):
+            arr[i] = d
+        return arr
+
+    good = ObLayer(p, p, p, p, p, 64, 32, 0, 0)
+    ws, wsn = p, lib.ob_stack_workspace_size()
+    assert lib.ob_linear_stack(layers(good), 1, 17, ws, wsn, None) == SHAPE       # M > 16
+    assert lib.ob_linear_stack(layers(good), 0, 4, ws, wsn, None) == OK           # no layers
+    assert lib.ob_linear_stack(layers(good), 1, 0, ws, wsn, None) == OK           # no tokens
+    assert lib.ob_linear_stack(None, 1, 4, ws, wsn, None) == NULL
+    assert lib.ob_linear_stack(layers(good), 1, 4, None, wsn, None) == NULL
+    assert lib.ob_linear_stack(layers(good), 1, 4, bad, wsn, None) == ALIGN
+    assert lib.ob_linear_stack(layers(good), 1, 4, ws, 4, None) == WS
+    assert lib.ob_linear_stack(layers(good, ObLayer(p, p, p, p, p, 48, 32, 0, 1)), 2, 4, ws, wsn, None) == SHAPE
+    assert lib.ob_linear_stack(layers(ObLayer(p, p, p, p, p, 64, 0, 0, 0)), 1, 4, ws, wsn, None) == SHAPE
+    assert lib.ob_linear_stack(layers(ObLayer(p, p, p, p, p, 64, 32, 5, 0)), 1, 4, ws, wsn, None) == UNSUP
+    assert lib.ob_linear_stack(layers(ObLayer(p, None, p, p, p, 64, 32, 0, 0)), 1, 4, ws, wsn, None) == NULL
+    assert lib.ob_linear_stack(layers(ObLayer(p, p, p, bad, p, 64, 32, 0, 0)), 1, 4, ws, wsn, None) == ALIGN
+    # a null input scale is allowed (no scale); the next check that fails is the device context
+    st = lib.ob_linear_stack(layers(ObLayer(p, p, p, None, p, 64, 32, 0, 0)), 1, 4, ws, wsn, None)
+    assert st not in (NULL, SHAPE, ALIGN, WS, UNSUP)
