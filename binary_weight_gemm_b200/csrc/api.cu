@@ -307,7 +307,8 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   // Few output tiles (small M x r): split the first product over K into fp32 partial
   // sums after T in the workspace, when the workspace holds them.
   const bool tc1 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > decode_max_m() && K <= sign_gemm_tc_max_k());
-  const int ks = tc1 ? dbf_split_k(M, r, c.num_sms) : 1;
+  const bool split = env_flag("OB_DBF_SPLIT", true);  // OB_DBF_SPLIT=0: neither product is split
+  const int ks = (tc1 && split) ? dbf_split_k(M, r, c.num_sms) : 1;
   const size_t part_off = dbf_t_bytes(M, r);
   if (ks > 1 && path != OB_PATH_TC_DECODE && ws_bytes >= part_off + (size_t)ks * (size_t)M * (size_t)r * 4) {
     g1.l2_prefetch = 0;
@@ -318,10 +319,16 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   }
   if (st != OB_OK) return st;
   SignGemmArgs g2{T, M, r, SA_packed, N, nullptr, a, Y, N, y_dtype};
-  // The second product splits the same way when the region after T also holds its
-  // partial sums (the first product's are consumed before it runs).
+  // The second product (K = r) splits the same way when the region after T also holds
+  // its partial sums (the first product's are consumed before it runs), unless the
+  // CTA-pair kernel takes it and r < 4096: measured at M = 512 on B200, r = 2048
+  // unsplit on the pair kernel 42.6 us per layer against 44.7 split, r = 4704 split
+  // 64.4 against 67.6 unsplit.
   const bool tc2 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > decode_max_m() && r <= sign_gemm_tc_max_k());
-  const int ks2 = tc2 && M > decode_max_m() ? tc_split_k(M, N, c.num_sms) : 1;
+  const bool pair2 = env_flag("OB_TC2", true) && sign_gemm_tc2_supported(g2) && r < 4096;
+  const int ks2 = (tc2 && split && env_flag("OB_DBF_SPLIT2", !pair2) && M > decode_max_m())
+                      ? tc_split_k(M, N, c.num_sms)
+                      : 1;
   if (ks2 > 1 && ws_bytes >= part_off + (size_t)ks2 * (size_t)M * (size_t)N * 4)
     return status_of(launch_sign_gemm_tc_splitk(
         g2, ks2, reinterpret_cast<float*>(static_cast<char*>(workspace) + part_off), c));
