@@ -4,7 +4,9 @@
 // "proposition 1"); a decoder applies such layers one after another, a layer
 // reading the output of an earlier one.  Launched one kernel per layer, every
 // dependent layer pays a launch and a drain; here one cooperative grid walks the
-// whole list:
+// whole list.  This file holds the warp-level MMA form (any M <= 16) and the
+// launcher, which takes the table-lookup form of linear_stack_lut.cu instead for
+// one token when its shared-memory staging fits.  The MMA form:
 //  * A layer flagged as reading an earlier layer's output waits at a grid-wide
 //    barrier; the layers between two barriers run back to back.
 //  * A layer's rows are split into 32-row blocks dealt to the CTAs round robin,
@@ -22,78 +24,12 @@
 #include <cstring>
 
 #include "mma_decode_block.cuh"
+#include "stack_common.cuh"
 
 namespace ob {
 namespace {
 
 using namespace mmad;
-
-struct StackLayer {
-  const uint16_t* X;
-  const uint32_t* S;
-  const float* iscale;
-  const float* oscale;
-  void* Y;
-  int64_t K, N;
-  int32_t y_dtype;
-  int32_t barrier;  // wait for every earlier layer of the list before this one
-  int32_t nb;       // 32-row blocks: ceil(N / 32)
-  int32_t vec;      // the sign rows allow 16-byte copies
-};
-
-constexpr int kStackMaxLayers = 384;  // 384 x 72 B of kernel parameters
-
-struct StackParams {
-  int n;
-  int64_t M;
-  unsigned* bar;  // [0] arrivals, [1] abort
-  unsigned* err;
-  StackLayer L[kStackMaxLayers];
-};
-
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// All CTAs arrive; returns false (on every thread of the CTA) if the wait ran out
-// or another CTA aborted.
-__device__ bool grid_barrier(unsigned* bar, unsigned target, unsigned* err, int* s_ok) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();  // this CTA's outputs before its arrival
-    atomicAdd(bar, 1u);
-    int ok = 1;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-      if (ld_acquire_gpu(bar) >= target) break;
-      if ((it & 31u) == 0u) {
-        if (ld_acquire_gpu(bar + 1) != 0u) {
-          ok = 0;
-          break;
-        }
-        if (globaltimer_ns() - t0 > OB_WAIT_LIMIT_NS || it > (1u << 30)) {
-          record_error(err, OB_DEVERR_TIMEOUT);
-          atomicExch(bar + 1, 1u);
-          ok = 0;
-          break;
-        }
-      }
-    }
-    __threadfence();
-    *s_ok = ok;
-  }
-  __syncthreads();
-  return *s_ok != 0;
-}
-
-// The first layer index after the barrier group that starts at l.
-__device__ __forceinline__ int group_end(const StackParams& p, int l) {
-  int e = l + 1;
-  while (e < p.n && !p.L[e].barrier) ++e;
-  return e;
-}
 
 // First block of a layer dealt to CTA c when the group's round robin is at `off`.
 __device__ __forceinline__ int first_block(int c, int off, int G) {
@@ -183,7 +119,8 @@ cudaError_t launch_stack_tok(const StackParams& prm, const LaunchCtx& c) {
 
 int stack_max_layers_per_launch() { return kStackMaxLayers; }
 
-cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c) {
+cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c,
+                              bool allow_lut) {
   if (n == 0 || M == 0) return cudaSuccess;
   static_assert(sizeof(StackParams) <= 32000, "kernel parameters");
   StackParams* prm = new StackParams;
@@ -204,7 +141,10 @@ cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, un
     }
     e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned), c.stream);
     if (e != cudaSuccess) break;
-    e = M == 1 ? launch_stack_tok<1>(*prm, c) : (M <= 8 ? launch_stack_tok<8>(*prm, c) : launch_stack_tok<16>(*prm, c));
+    if (M == 1 && allow_lut && stack_lut_fits(*prm, c.num_sms))
+      e = launch_stack_lut(*prm, c);
+    else
+      e = M == 1 ? launch_stack_tok<1>(*prm, c) : (M <= 8 ? launch_stack_tok<8>(*prm, c) : launch_stack_tok<16>(*prm, c));
   }
   delete prm;
   return e;

@@ -77,8 +77,10 @@ struct StackLayerHost {
   int barrier;          // reads an output of an earlier layer of the list
 };
 // Runs the list (M <= 16) as cooperative launches of at most stack_max_layers_per_launch()
-// layers; bar: 8 bytes of device memory (zeroed by the launcher).
-cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c);
+// layers; bar: 8 bytes of device memory (zeroed by the launcher).  allow_lut: at M = 1,
+// use the table-lookup kernel where its staging fits.
+cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c,
+                              bool allow_lut);
 int stack_max_layers_per_launch();
 
 // Z = LayerNorm(Y) per row of the M x N matrix Y (row stride ld elements), in place.

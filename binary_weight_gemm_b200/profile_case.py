@@ -3,12 +3,18 @@
     python -m binary_weight_gemm_b200.profile_case decode --m 16 --reps 40
     python -m binary_weight_gemm_b200.profile_case prefill --reps 6
     python -m binary_weight_gemm_b200.profile_case dbf --m 512 --reps 6
+    python -m binary_weight_gemm_b200.profile_case stack --m 1 --blocks 8 --reps 5
+    python -m binary_weight_gemm_b200.profile_case stack --m 1 --chain 128 --reps 5
 
 The workloads are the benchmark's: OneBit 4096 x 4096 decode at M tokens, OneBit
-prefill X 2048 x 4096 -> 11008, DBF K = N = 4096 with r = 2048.  Weights come from
-the library's own pack and SVID of the seeded W.  Several distinct weight / input
-sets rotate so that their total exceeds the 126 MB L2 (DRAM counters then count
-real traffic), while the device holds a few hundred MB at most.  Prints one JSON
+prefill X 2048 x 4096 -> 11008, DBF K = N = 4096 with r = 2048, and the layer stack:
+one ob_linear_stack over `blocks` 7B-shaped blocks (q, k, v, o 4096 -> 4096; gate, up
+4096 -> 11008; down 11008 -> 4096), or with --chain C over C chained 1024 -> 1024
+layers (one barrier group each: the per-group cost with little work in it).  Weights
+come from the library's own pack and SVID of the seeded W.  Several distinct weight /
+input sets rotate so that their total exceeds the 126 MB L2 (DRAM counters then count
+real traffic), while the device holds a few hundred MB at most; every stack layer has
+its own copy of the weights.  Prints one JSON
 line with the mean time per call measured with CUDA events (not meaningful under
 a profiler).
 """
@@ -35,9 +41,11 @@ def _bf16(x_bits: np.ndarray, dev) -> torch.Tensor:
 
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("case", choices=("decode", "prefill", "dbf"))
-    ap.add_argument("--m", type=int, default=None, help="tokens (decode default 16, dbf default 512)")
+    ap.add_argument("case", choices=("decode", "prefill", "dbf", "stack"))
+    ap.add_argument("--m", type=int, default=None, help="tokens (decode default 16, dbf default 512, stack 1)")
     ap.add_argument("--reps", type=int, default=6)
+    ap.add_argument("--blocks", type=int, default=8, help="stack: 7B-shaped blocks")
+    ap.add_argument("--chain", type=int, default=0, help="stack: chained 1024 -> 1024 layers instead")
     args = ap.parse_args(argv)
     dev = torch.device("cuda", 0)
     torch.cuda.init()
@@ -58,6 +66,38 @@ def main(argv=None) -> None:
         def call(i):
             X, P, a, b, Y = sets[i % n_sets]
             ops.ob_linear(X, P, a, b, out=Y)
+    elif args.case == "stack":
+        M = args.m or 1
+        if args.chain:
+            shapes = [(f"l{i}", 1024, 1024) for i in range(args.chain)]
+        else:
+            shapes = [(n, K, N) for _ in range(args.blocks)
+                      for n, K, N in (("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+                                      ("gate", 4096, 11008), ("up", 4096, 11008), ("down", 11008, 4096))]
+        base = {}
+        for _, K, N in shapes:
+            if (K, N) not in base:
+                W = torch.from_numpy(synth.weights(7 + K % 97 + N % 89, N, K)).to(dev)
+                a0, b0, _, _, _ = ops.ob_svid_rank1(W)
+                base[(K, N)] = (ops.ob_pack_signs(W), a0, b0)
+                del W
+        X0 = _bf16(synth.activations(7, M, shapes[0][1])[0], dev)
+        spec, out, x = [], {}, X0
+        for i, (name, K, N) in enumerate(shapes):
+            P, a0, b0 = (t.clone() for t in base[(K, N)])
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            src = {"q": x, "k": x, "v": x, "o": out.get("q"), "gate": out.get("o"), "up": out.get("o"),
+                   "down": out.get("gate")}.get(name, x)
+            spec.append((src, P, a0, b0, Y, i > 0 and name not in ("k", "v", "up")))
+            out[name] = Y
+            if name in ("down",) or args.chain:
+                x = Y
+        desc = {"layers": len(spec), "blocks": 0 if args.chain else args.blocks}
+        ws = torch.zeros(ops.ob_stack_workspace_size(), dtype=torch.uint8, device=dev)
+        n_sets = 1
+
+        def call(i):
+            ops.ob_linear_stack(spec, M, workspace=ws)
     else:
         M, N, K, r = args.m or 512, 4096, 4096, 2048
         f = synth.dbf_factors(3, N, r, K)
@@ -83,7 +123,9 @@ def main(argv=None) -> None:
     e1.record()
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
-    print(json.dumps({"case": args.case, "M": M, "N": N, "K": K, "reps": args.reps, "sets": n_sets,
+    if args.case != "stack":
+        desc = {"N": N, "K": K}
+    print(json.dumps({"case": args.case, "M": M, **desc, "reps": args.reps, "sets": n_sets,
                       "us_per_call": e0.elapsed_time(e1) * 1e3 / args.reps}))
 
 

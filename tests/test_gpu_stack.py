@@ -1,8 +1,13 @@
 """GPU parity of ob_linear_stack (a list of OneBit layers in one persistent launch).
 
 Every layer is checked against the fp64 oracle on the bf16 input it actually
-received (its X, possibly an earlier layer's Y), with the GEMM tolerances.
+received (its X, possibly an earlier layer's Y), with the GEMM tolerances.  At one
+token the library runs the table-lookup kernel when every layer's K is a multiple
+of 128 (and the shares fit its staging buffer), else the warp-MMA kernel;
+OB_STACK_LUT=0 forces the latter.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -21,6 +26,17 @@ def ops():
     from binary_weight_gemm_b200 import ops as _ops
     torch.cuda.init()
     return _ops
+
+
+@pytest.fixture
+def mma_form():
+    old = os.environ.get("OB_STACK_LUT")
+    os.environ["OB_STACK_LUT"] = "0"
+    yield
+    if old is None:
+        del os.environ["OB_STACK_LUT"]
+    else:
+        os.environ["OB_STACK_LUT"] = old
 
 
 def _cuda(x):
@@ -65,6 +81,33 @@ def test_stack_chain(ops, M):
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
     _check(host, [(s[0], s[4]) for s in spec], f"chain M={M}")
+
+
+def test_stack_chain_mma_form_one_token(ops, mma_form):
+    test_stack_chain(ops, 1)
+
+
+def test_stack_lut_passes_and_segments(ops):
+    # One token.  Group 1 (all read X0, K = 128): 60 layers of 32 rows (more layers than a
+    # CTA's segment slots, so the host checks every CTA's share; the first writes fp32),
+    # one of 30000 rows (about 203 rows per CTA: two passes of the table kernel), one of
+    # 1152 rows.  Group 2 reads the 1152-wide output: K = 1152 is one full 1024-k chunk
+    # and a 128-k tail; 300 rows, no input scale.
+    M = 1
+    X0 = _x(synth.activations(270, M, 128)[0])
+    shapes = [(32, 128)] * 60 + [(30000, 128), (1152, 128), (300, 1152)]
+    host, spec = [], []
+    for i, (N, K) in enumerate(shapes):
+        last = i == len(shapes) - 1
+        W, a, b = _layer(300 + i, N, K, scale_in=not last)
+        host.append((W, a, b))
+        Y = torch.empty((M, N), dtype=torch.float32 if i == 0 else torch.bfloat16, device="cuda")
+        X = spec[-1][4] if last else X0
+        spec.append((X, ops.ob_pack_signs(_cuda(W)), _cuda(a), None if last else _cuda(b), Y, last))
+    ops.ob_linear_stack(spec, M)
+    torch.cuda.synchronize()
+    assert ops.ob_last_device_error() == 0
+    _check(host, [(sp[0], sp[4]) for sp in spec], "lut stack")
 
 
 @pytest.mark.parametrize("M", [1, 5, 16])
@@ -154,8 +197,20 @@ def test_stack_in_cuda_graph(ops):
     _check(host, [(sp[0], sp[4]) for sp in spec], "graph stack")
 
 
-@pytest.mark.parametrize("M", [1, 16])
-def test_stack_7b_block(ops, M):
+@pytest.mark.parametrize("M,lut", [(1, True), (1, False), (16, True)], ids=["M1", "M1-mma", "M16"])
+def test_stack_7b_block(ops, M, lut):
+    old = os.environ.get("OB_STACK_LUT")
+    os.environ["OB_STACK_LUT"] = "1" if lut else "0"
+    try:
+        _stack_7b_block(ops, M)
+    finally:
+        if old is None:
+            del os.environ["OB_STACK_LUT"]
+        else:
+            os.environ["OB_STACK_LUT"] = old
+
+
+def _stack_7b_block(ops, M):
     # One 7B-shaped block: q, k, v, o (4096 -> 4096), gate, up (4096 -> 11008), down (11008 -> 4096).
     Wq, aq, bq, _ = oracle_svid(1, 4096, 4096)
     Wg, ag, bg, _ = oracle_svid(5, 11008, 4096)
