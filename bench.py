@@ -642,11 +642,11 @@ def run_stack(args, world, rank, local):
             pgraphs[m] = torch.cuda.CUDAGraph()
             with torch.cuda.graph(pgraphs[m], stream=stream):
                 ops.ob_linear_stack(specs[m], m, workspace=ws, stream=stream)
-        # At one token the library runs the table-lookup stack kernel; the warp-MMA form
-        # (OB_STACK_LUT=0) is timed beside it.
+        # The table-lookup stack kernel (OB_STACK_LUT=1, one token) is timed beside the
+        # default warp-MMA form.
         mgraphs = {}
         old = os.environ.get("OB_STACK_LUT")
-        os.environ["OB_STACK_LUT"] = "0"
+        os.environ["OB_STACK_LUT"] = "1"
         try:
             ops.ob_linear_stack(specs[1], 1, workspace=ws, stream=stream)
             stream.synchronize()
@@ -666,7 +666,7 @@ def run_stack(args, world, rank, local):
 
     ms_max, ms, clocks = _timed(step, args, world, stream, local)
     per_m = {}
-    for mode, gs in (("persistent", pgraphs), ("per_call", graphs), ("persistent_mma", mgraphs)):
+    for mode, gs in (("persistent", pgraphs), ("per_call", graphs), ("persistent_lut", mgraphs)):
         for m in gs:
             reps = max(3, args.steps // 2)
             with torch.cuda.stream(stream):
@@ -697,8 +697,8 @@ def run_stack(args, world, rank, local):
                        "layers_per_token": calls, "weights_mb": wbytes / 1e6,
                        "l2": f"inputs larger than L2: {blocks * 7} distinct weight buffers ({wbytes / 1e6:.0f} MB)",
                        "graph": "one CUDA graph per token and M holding one ob_linear_stack (persistent, "
-                                "grid barriers between dependent layers; at M = 1 the table-lookup kernel, "
-                                "persistent_mma_M1 the warp-MMA form); per_call_* times one ob_linear "
+                                "grid barriers between dependent layers; warp-MMA kernel, "
+                                "persistent_lut_M1 the table-lookup kernel); per_call_* times one ob_linear "
                                 "per layer in a graph with programmatic dependent launch",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "per_m": per_m,

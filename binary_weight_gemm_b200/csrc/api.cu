@@ -258,7 +258,7 @@ ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M, void*
   ob_status st = make_ctx(stream, &c);
   if (st != OB_OK) return st;
   return status_of(launch_sign_stack(host.data(), n_layers, M, static_cast<unsigned*>(workspace), c,
-                                     env_flag("OB_STACK_LUT", true)));
+                                     env_flag("OB_STACK_LUT", false)));
 }
 
 // Bytes of the bf16 intermediate T: the smallest workspace dbf_linear accepts.

@@ -4,9 +4,10 @@
 // "proposition 1"); a decoder applies such layers one after another, a layer
 // reading the output of an earlier one.  Launched one kernel per layer, every
 // dependent layer pays a launch and a drain; here one cooperative grid walks the
-// whole list.  This file holds the warp-level MMA form (any M <= 16) and the
-// launcher, which takes the table-lookup form of linear_stack_lut.cu instead for
-// one token when its shared-memory staging fits.  The MMA form:
+// whole list.  This file holds the warp-level MMA form (any M <= 16, the default)
+// and the launcher, which takes the table-lookup form of linear_stack_lut.cu instead
+// for one token when the caller asks for it and its shared-memory staging fits.
+// The MMA form:
 //  * A layer flagged as reading an earlier layer's output waits at a grid-wide
 //    barrier; the layers between two barriers run back to back.
 //  * A layer's rows are split into 32-row blocks dealt to the CTAs round robin,

@@ -27,8 +27,12 @@
 //    scale vectors of the next group are prefetched into L2 with its sign rows.
 //  * Warp w holds the partial sums of rows w, w+16, ... (12 per warp, 192 rows per
 //    pass of a segment) in registers across the chunks.
-// The launcher uses this form only when every CTA's share of every group fits one
-// staging buffer (stack_lut_fits); otherwise the MMA form runs.
+// The launcher uses this form only when asked (OB_STACK_LUT=1) and every CTA's share
+// of every group fits one staging buffer (stack_lut_fits); otherwise the MMA form runs.
+// Measured on B200 for one token through 32 blocks of 7B-shaped layers: 2118 us per
+// token against 1769 us for the MMA form.  DRAM traffic equals the packed weights (no
+// re-reads); the largest stall is the CTA barrier (one per 1024-k chunk, load imbalance
+// between warps when a CTA holds few rows, and the grid barrier).
 #include <algorithm>
 #include <cstring>
 

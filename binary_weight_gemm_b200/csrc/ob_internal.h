@@ -78,7 +78,8 @@ struct StackLayerHost {
 };
 // Runs the list (M <= 16) as cooperative launches of at most stack_max_layers_per_launch()
 // layers; bar: 8 bytes of device memory (zeroed by the launcher).  allow_lut: at M = 1,
-// use the table-lookup kernel where its staging fits.
+// use the table-lookup kernel where its staging fits (OB_STACK_LUT=1; measured slower
+// than the warp-MMA form on the 7B-shaped stack, so off by default).
 cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c,
                               bool allow_lut);
 int stack_max_layers_per_launch();

@@ -222,6 +222,11 @@ OB_API size_t ob_stack_workspace_size(void);
  *              concurrently running ob_linear_stack.
  * Weights and scales must not be outputs of layers of the same list.  Validation of
  * every descriptor happens before anything is launched.  Asynchronous.
+ * Kernel: warp-level MMA blocks by default; with the environment variable
+ * OB_STACK_LUT=1 and M == 1, a table-lookup kernel that stages each CTA's sign rows
+ * in shared memory (used when every K is a multiple of 128 and every CTA's share of
+ * a group fits 80 KB; otherwise the default runs).  Same results within the
+ * tolerances; the default was the faster of the two on 7B-shaped layers.
  */
 OB_API ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M,
                           void* workspace, size_t ws_bytes, void* stream);

@@ -1,10 +1,10 @@
 """GPU parity of ob_linear_stack (a list of OneBit layers in one persistent launch).
 
 Every layer is checked against the fp64 oracle on the bf16 input it actually
-received (its X, possibly an earlier layer's Y), with the GEMM tolerances.  At one
-token the library runs the table-lookup kernel when every layer's K is a multiple
-of 128 (and the shares fit its staging buffer), else the warp-MMA kernel;
-OB_STACK_LUT=0 forces the latter.
+received (its X, possibly an earlier layer's Y), with the GEMM tolerances.  The
+warp-MMA kernel is the default; at one token OB_STACK_LUT=1 selects the table-lookup
+kernel where every layer's K is a multiple of 128 and the shares fit its staging
+buffer (the tests marked "lut" below set it).
 """
 import os
 
@@ -29,9 +29,9 @@ def ops():
 
 
 @pytest.fixture
-def mma_form():
+def lut_form():
     old = os.environ.get("OB_STACK_LUT")
-    os.environ["OB_STACK_LUT"] = "0"
+    os.environ["OB_STACK_LUT"] = "1"
     yield
     if old is None:
         del os.environ["OB_STACK_LUT"]
@@ -83,11 +83,15 @@ def test_stack_chain(ops, M):
     _check(host, [(s[0], s[4]) for s in spec], f"chain M={M}")
 
 
-def test_stack_chain_mma_form_one_token(ops, mma_form):
+def test_stack_chain_lut_form_one_token(ops, lut_form):
     test_stack_chain(ops, 1)
 
 
-def test_stack_lut_passes_and_segments(ops):
+def test_stack_dbf_lut_form_one_token(ops, lut_form):
+    test_stack_dbf(ops, 1)
+
+
+def test_stack_lut_passes_and_segments(ops, lut_form):
     # One token.  Group 1 (all read X0, K = 128): 60 layers of 32 rows (more layers than a
     # CTA's segment slots, so the host checks every CTA's share; the first writes fp32),
     # one of 30000 rows (about 203 rows per CTA: two passes of the table kernel), one of
