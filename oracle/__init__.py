@@ -15,25 +15,31 @@ Everything is plain NumPy in float64, written from the definitions on the pages:
 * DBF, from "Addition is almost all you need: Compressing large language models
   with double binary factorization" (gist.science, section "Methodologie:
   Double Binary Factorization (DBF)"): the factorised weight and its inference
-  chain.
+  chain; and, in the submodule ``oracle.dbf_factorize``, the factorisation
+  W -> (S_A, S_B, a, m, b) by alternating ADMM steps with an SVID projection
+  ("Optimalisatie en Training").
 
 The linear layers are computed in the DIRECT form -- the approximated weight
 matrix is materialised and then multiplied -- not in the factorised order the
 kernels use, so that agreement is evidence rather than repetition.
 
-Parity status: every public function here is pinned by tests under
-``tests/test_oracle_*.py`` against hand-computed worked examples
-(``tests/golden/``), closed forms, special cases and brute force.  None is
-"parity unpinned".
+Parity status: every public function of ``oracle.onebit`` and ``oracle.dbf`` is
+pinned by tests under ``tests/test_oracle_*.py`` against hand-computed worked
+examples (``tests/golden/``), closed forms, special cases and brute force.  In
+``oracle.dbf_factorize`` the steps are pinned the same way (projection, ADMM
+least-squares steps, scale refits), but the factorisation loop as a whole is
+"parity unpinned": the page names a heuristic without giving its steps, so only
+exact recovery and properties of the result can be checked.
 """
 from .onebit import (sign_pm1, pack_signs, unpack_signs, rank1_svd, svid_rank1,
                      onebit_weight, onebit_linear, onebit_linear_packed,
                      onebit_linear_prop1, layernorm, onebit_linear_ln, LN_EPS)
 from .dbf import dbf_weight, dbf_linear, dbf_linear_chain
+from . import dbf_factorize
 
 __all__ = [
     "sign_pm1", "pack_signs", "unpack_signs", "rank1_svd", "svid_rank1",
     "onebit_weight", "onebit_linear", "onebit_linear_packed", "onebit_linear_prop1",
     "layernorm", "onebit_linear_ln", "LN_EPS",
-    "dbf_weight", "dbf_linear", "dbf_linear_chain",
+    "dbf_weight", "dbf_linear", "dbf_linear_chain", "dbf_factorize",
 ]

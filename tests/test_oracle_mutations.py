@@ -3,12 +3,17 @@
 Each case takes the oracle's source, plants one mistake by a text replacement (a
 reversed bit order, a wrong sign threshold, a dropped |.|, the smallest instead of
 the largest singular triple, a flipped unpack polarity, a dropped middle or input
-scale, reversed columns, an unbiased variance, a missing mean subtraction),
-executes the result as fresh in-memory
-modules (nothing is written to disk) and runs a compact set of the pins against
-it: the hand-worked fixtures under tests/golden/, the pack/unpack round trip,
-Proposition 2's closed form and the DBF chain against the direct form.  Every
-mutant must fail at least one pin; the unmodified oracle must pass all of them.
+scale, reversed columns, an unbiased variance, a missing mean subtraction; in the
+factorisation a dropped ADMM penalty or pull, a wrong dual sign, dropped signs in
+the projection, half of the middle scale lost, a matrix instead of a Hadamard
+product in the Gram matrix, a biased refit), executes the result as fresh
+in-memory modules (nothing is written to disk) and runs a compact set of the pins
+against it: the hand-worked fixtures under tests/golden/, the pack/unpack round
+trip, Proposition 2's closed form, the DBF chain against the direct form, the
+projection's closed-form error, the ADMM steps and scale refits against library
+least squares, exact recovery of a rank-1 DBF weight and the low-rank property.
+Every mutant must fail at least one pin; the unmodified oracle must pass all of
+them.
 """
 import json
 import os
@@ -21,21 +26,30 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
+# dbf_factorize.py takes these names from its sibling modules; the loader strips the
+# relative imports and hands it the (possibly mutated) versions loaded before it.
+_SIBLING_IMPORTS = "from .dbf import dbf_weight\nfrom .onebit import sign_pm1, svid_rank1\n"
+
+
 def _load(mutation=None):
     """The oracle's public functions from its sources, with one optional (file, old, new) replacement.
 
     onebit.py and dbf.py import only numpy, so each executes on its own.
     """
     ns = types.SimpleNamespace()
-    for fname in ("onebit.py", "dbf.py"):
+    for fname in ("onebit.py", "dbf.py", "dbf_factorize.py"):
         src = open(os.path.join(ROOT, "oracle", fname), encoding="utf-8").read()
         if mutation and mutation[0] == fname:
             assert mutation[1] in src, mutation
             src = src.replace(mutation[1], mutation[2], 1)
         mod = types.ModuleType("oracle_" + fname[:-3])
+        if fname == "dbf_factorize.py":
+            assert _SIBLING_IMPORTS in src
+            src = src.replace(_SIBLING_IMPORTS, "")
+            mod.__dict__.update(dbf_weight=ns.dbf_weight, sign_pm1=ns.sign_pm1, svid_rank1=ns.svid_rank1)
         exec(compile(src, "oracle/" + fname, "exec"), mod.__dict__)
         for k, v in vars(mod).items():
-            if not k.startswith("_"):
+            if not k.startswith("_") and not (fname == "dbf_factorize.py" and hasattr(ns, k)):
                 setattr(ns, k, v)
     return ns
 
@@ -109,9 +123,61 @@ def _pins(o):
         g = _golden("layernorm_4.json")
         return np.allclose(o.layernorm(np.array(g["Y"]), eps=g["eps"]), g["Z"], atol=1e-12)
 
+    def projection_closed_form():
+        M = np.random.default_rng(4).standard_normal((7, 5))
+        Z = o.structured(*o.svid_project(M))
+        lam = np.linalg.eigvalsh(np.abs(M).T @ np.abs(M))[-1]
+        return abs(np.linalg.norm(M - Z) ** 2 - (np.linalg.norm(M) ** 2 - lam)) < 1e-9
+
+    def admm_step_lstsq():
+        rng = np.random.default_rng(5)
+        W, ZA, UA = rng.standard_normal((4, 7)), rng.standard_normal((4, 3)), rng.standard_normal((4, 3))
+        ZB, UB = rng.standard_normal((3, 7)), rng.standard_normal((3, 7))
+        rho = 0.6
+        A = o.admm_left_step(W, ZB, ZA, UA, rho)
+        DA = np.vstack([ZB.T, np.sqrt(rho) * np.eye(3)])
+        ok = all(np.allclose(A[n], np.linalg.lstsq(DA, np.concatenate([W[n], np.sqrt(rho) * (ZA - UA)[n]]),
+                                                    rcond=None)[0]) for n in range(4))
+        B = o.admm_right_step(W, ZA, ZB, UB, rho)
+        DB = np.vstack([ZA, np.sqrt(rho) * np.eye(3)])
+        ok &= all(np.allclose(B[:, k], np.linalg.lstsq(DB, np.concatenate([W[:, k], np.sqrt(rho) * (ZB - UB)[:, k]]),
+                                                        rcond=None)[0]) for k in range(7))
+        return ok
+
+    def refit_lstsq():
+        rng = np.random.default_rng(6)
+        W = rng.standard_normal((5, 6))
+        SA, SB = np.sign(rng.standard_normal((5, 3))), np.sign(rng.standard_normal((3, 6)))
+        a, m, b = rng.uniform(0.5, 2, 5), rng.uniform(0.5, 2, 3), rng.uniform(0.5, 2, 6)
+        D = np.stack([np.outer(a * SA[:, j], SB[j] * b).ravel() for j in range(3)], axis=1)
+        ok = np.allclose(o.refit_m(W, SA, SB, a, b), np.linalg.lstsq(D, W.ravel(), rcond=None)[0])
+        R = SA @ np.diag(m) @ SB @ np.diag(b)
+        ok &= np.allclose(o.refit_a(W, SA, SB, m, b), (W * R).sum(1) / (R * R).sum(1))
+        C = np.diag(a) @ SA @ np.diag(m) @ SB
+        ok &= np.allclose(o.refit_b(W, SA, SB, a, m), (W * C).sum(0) / (C * C).sum(0))
+        return ok
+
+    def factorize_exact_rank1():
+        rng = np.random.default_rng(7)
+        W = o.dbf_weight(np.sign(rng.standard_normal((6, 1))), np.sign(rng.standard_normal((1, 8))),
+                         rng.uniform(0.2, 2, 6), rng.uniform(0.5, 2, 1), rng.uniform(0.2, 2, 8))
+        res = o.dbf_factorize(W, 1, sweeps=2, refit_rounds=0)
+        return res["error"] <= 1e-10 * np.linalg.norm(W)
+
+    def factorize_low_rank():
+        rng = np.random.default_rng(0)
+        N, K = 96, 128
+        W = rng.standard_normal((N, 8)) @ rng.standard_normal((8, K)) * 0.01 + 0.001 * rng.standard_normal((N, K))
+        a, b, _ = o.svid_rank1(W)
+        e1 = np.linalg.norm(W - o.onebit_weight(o.sign_pm1(W), a, b))
+        return o.dbf_factorize(W, N * K // (N + K))["error"] < 0.6 * e1
+
     for name, fn in (("pack_golden", pack_golden), ("pack_roundtrip", pack_roundtrip), ("svid_golden", svid_golden),
                      ("prop2_closed_form", prop2_closed_form), ("linear_golden", linear_golden),
-                     ("dbf_golden", dbf_golden), ("dbf_chain", dbf_chain), ("layernorm_golden", layernorm_golden)):
+                     ("dbf_golden", dbf_golden), ("dbf_chain", dbf_chain), ("layernorm_golden", layernorm_golden),
+                     ("projection_closed_form", projection_closed_form), ("admm_step_lstsq", admm_step_lstsq),
+                     ("refit_lstsq", refit_lstsq), ("factorize_exact_rank1", factorize_exact_rank1),
+                     ("factorize_low_rank", factorize_low_rank)):
         check(name, fn)
     return failed
 
@@ -130,6 +196,13 @@ MUTATIONS = [
     ("onebit.py", "var = ((Y - mean) ** 2).mean(axis=1, keepdims=True)",
      "var = ((Y - mean) ** 2).sum(axis=1, keepdims=True) / (Y.shape[1] - 1)"),              # unbiased variance
     ("onebit.py", "return (Y - mean) / np.sqrt(var + eps)", "return Y / np.sqrt(var + eps)"),  # no mean removal
+    ("dbf_factorize.py", "G = ZB @ ZB.T + rho * np.eye(r)", "G = ZB @ ZB.T"),                  # penalty dropped
+    ("dbf_factorize.py", "R = W @ ZB.T + rho * (ZA - UA)", "R = W @ ZB.T + rho * (ZA + UA)"),  # dual sign
+    ("dbf_factorize.py", "R = ZA.T @ W + rho * (ZB - UB)", "R = ZA.T @ W"),                   # right pull dropped
+    ("dbf_factorize.py", "return sign_pm1(M), u, v", "return sign_pm1(np.abs(M)), u, v"),      # signs dropped
+    ("dbf_factorize.py", "a, m, b = uA, vA * uB, vB", "a, m, b = uA, vA, vB"),                 # middle scale half lost
+    ("dbf_factorize.py", "G = (P.T @ P) * (Q @ Q.T)", "G = (P.T @ P) @ (Q @ Q.T)"),             # Gram product
+    ("dbf_factorize.py", "den = (C * C).sum(axis=0)", "den = (C * C).sum(axis=0) + 1.0"),      # biased b refit
 ]
 
 
