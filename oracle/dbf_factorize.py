@@ -23,7 +23,10 @@ notes):
   rank-1 SVID of |M| (the same construction as OneBit's, applied to a factor).
 * Initialisation: the rank-r truncated SVD W ≈ U_r Σ_r V_r^T split evenly,
   A = U_r Σ_r^(1/2), B = Σ_r^(1/2) V_r^T (zero columns/rows past min(N, K)),
-  then Z_A, Z_B their projections and the scaled duals zero.
+  then Z_A, Z_B their projections and the scaled duals zero.  Alternatively (the
+  start a GPU can run without an SVD) a sketch: A = W Ω for a given K x r matrix Ω
+  (random numbers drawn by the caller), B = argmin ||W - A B|| with a ridge of
+  1e-6 * trace(A^T A) / r.
 * One sweep: `admm_iters` ADMM steps on the left factor with Z_B fixed, then as
   many on the right factor with Z_A fixed.  An ADMM step on the left factor for
   min ||W - A Z_B||_F^2 subject to A in the set, with the split A = Z_A and the
@@ -84,6 +87,17 @@ def dbf_init(W: np.ndarray, r: int) -> tuple[np.ndarray, np.ndarray]:
     return A, B
 
 
+def dbf_init_sketch(W: np.ndarray, omega: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """A = W Ω (N x r); B = (A^T A + eps I)^-1 A^T W with eps = 1e-6 trace(A^T A) / r."""
+    W = np.asarray(W, dtype=np.float64)
+    A = W @ np.asarray(omega, dtype=np.float64)
+    r = A.shape[1]
+    G = A.T @ A
+    eps = 1e-6 * float(np.trace(G)) / r
+    B = np.linalg.solve(G + eps * np.eye(r), A.T @ W)
+    return A, B
+
+
 def admm_left_step(W, ZB, ZA, UA, rho):
     """argmin_A ||W - A ZB||_F^2 + rho ||A - ZA + UA||_F^2 = (W ZB^T + rho (ZA - UA)) (ZB ZB^T + rho I)^-1."""
     r = ZB.shape[0]
@@ -136,17 +150,19 @@ def dbf_error(W, S_A, S_B, a, m, b) -> float:
 
 
 def dbf_factorize(W: np.ndarray, r: int, sweeps: int = 20, admm_iters: int = 3, rho_rel: float = 1.0,
-                  refit_rounds: int = 2) -> dict:
+                  refit_rounds: int = 2, omega: np.ndarray | None = None) -> dict:
     """Factorise W (N x K) as diag(a) S_A diag(m) S_B diag(b) with middle dimension r.
 
+    omega: None for the truncated-SVD start, or a K x r matrix for the sketch start.
     Returns a dict with S_A (N x r, +/-1), S_B (r x K, +/-1), a (N), m (r), b (K), all
     float64; "history": ||W - Z_A Z_B||_F after every sweep; "best": the smallest of
-    them (the iterate kept); "error": the error after the scale refit.
+    the start's error and them (the iterate kept); "error": the error after the scale
+    refit.
     """
     W = np.asarray(W, dtype=np.float64)
     if W.ndim != 2 or r < 1:
         raise ValueError("W must be a matrix and r >= 1")
-    A, B = dbf_init(W, r)
+    A, B = dbf_init(W, r) if omega is None else dbf_init_sketch(W, omega)
     pa = svid_project(A)
     pb = svid_project(B)
     ZA, ZB = structured(*pa), structured(*pb)

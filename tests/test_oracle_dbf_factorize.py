@@ -121,6 +121,42 @@ def test_exact_recovery_of_a_rank1_dbf_weight(refit_rounds):
         assert res["error"] <= 1e-10 * np.linalg.norm(W)
 
 
+def test_sketch_start_recovers_a_rank1_dbf_weight():
+    # W Ω spans W's column space when W has rank 1, so the sketch start is exact too.
+    rng = _rng(85)
+    N, K, r = 9, 13, 4
+    W = oracle.dbf_weight(_pm1(rng, (N, 1)), _pm1(rng, (1, K)), rng.uniform(0.2, 2, N), rng.uniform(0.5, 2, 1),
+                          rng.uniform(0.2, 2, K))
+    A, B = F.dbf_init_sketch(W, rng.standard_normal((K, r)))
+    assert np.linalg.norm(W - A @ B) <= 1e-5 * np.linalg.norm(W)
+    res = F.dbf_factorize(W, r, sweeps=3, refit_rounds=0, omega=rng.standard_normal((K, r)))
+    assert res["error"] <= 1e-5 * np.linalg.norm(W)
+
+
+def test_sketch_start_solves_the_ridge_least_squares():
+    rng = _rng(86)
+    W, omega = rng.standard_normal((8, 11)), rng.standard_normal((11, 3))
+    A, B = F.dbf_init_sketch(W, omega)
+    assert np.allclose(A, W @ omega)
+    eps = 1e-6 * np.trace(A.T @ A) / 3
+    for k in range(11):
+        D = np.vstack([A, np.sqrt(eps) * np.eye(3)])
+        t = np.concatenate([W[:, k], np.zeros(3)])
+        assert np.allclose(B[:, k], np.linalg.lstsq(D, t, rcond=None)[0], atol=1e-10)
+
+
+def test_sketch_start_beats_onebit_on_a_low_rank_weight():
+    # 128 x 128 at r = 64: the same bits as OneBit, and r a multiple of the packed word.
+    rng = _rng(0)
+    N = K = 128
+    W = rng.standard_normal((N, 8)) @ rng.standard_normal((8, K)) * 0.01 + 0.001 * rng.standard_normal((N, K))
+    r = 64
+    a, b, _ = oracle.svid_rank1(W)
+    e_onebit = np.linalg.norm(W - oracle.onebit_weight(oracle.sign_pm1(W), a, b))
+    res = F.dbf_factorize(W, r, omega=np.random.default_rng(1).standard_normal((K, r)) / np.sqrt(K))
+    assert res["error"] < 0.6 * e_onebit
+
+
 def test_result_invariants():
     rng = _rng(90)
     N, K, r = 20, 28, 11
