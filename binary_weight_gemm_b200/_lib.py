@@ -48,6 +48,9 @@ SIGNATURES = {
     "dbf_linear_ex": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P, _P, _I, _P, _SZ, _I, _P]),
     "ob_selftest_timeout": (_I, [_U64, _P]),
     "dbf_linear_noalloc": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P, _P, _I, _P]),
+    "dbf_factorize_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "dbf_factorize": (_I, [_P, _I64, _I64, _I64, _P, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                           _P]),
 }
 DBF_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 

@@ -121,6 +121,9 @@ ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Largest N, K or r of dbf_factorize: its GEMM grid has one row of CTAs per 64 rows.
+constexpr int64_t kFactorizeMaxDim = (int64_t)1 << 22;
+
 }  // namespace
 }  // namespace ob
 
@@ -368,6 +371,33 @@ ob_status dbf_linear_noalloc(const void* X, int64_t M, int64_t K, const uint32_t
   }
   return dbf_linear_ex(X, M, K, SB_packed, r, m, SA_packed, N, a, b, Y, y_dtype, ptr,
                        (size_t)OB_DBF_NOALLOC_SCRATCH_BYTES, OB_PATH_AUTO, stream);
+}
+
+size_t dbf_factorize_workspace_size(int64_t N, int64_t K, int64_t r) {
+  if (N < 1 || K < 32 || r < 32 || K % 32 != 0 || r % 32 != 0) return 0;
+  if (N > kFactorizeMaxDim || K > kFactorizeMaxDim || r > kFactorizeMaxDim) return 0;
+  return dbf_factorize_workspace_bytes(N, K, r);
+}
+
+ob_status dbf_factorize(const float* W, int64_t N, int64_t K, int64_t r, const float* omega, int sweeps,
+                        int admm_iters, int cg_iters, float rho_rel, int refit_rounds, uint32_t* SA_packed,
+                        uint32_t* SB_packed, float* a, float* m, float* b, float* history, float* best,
+                        float* error, void* workspace, size_t ws_bytes, void* stream) {
+  if (N < 1 || K < 32 || r < 32 || K % 32 != 0 || r % 32 != 0) return OB_ERR_SHAPE;
+  if (N > kFactorizeMaxDim || K > kFactorizeMaxDim || r > kFactorizeMaxDim) return OB_ERR_SHAPE;
+  if (sweeps < 0 || sweeps > 100000 || admm_iters < 1 || admm_iters > 1000 || cg_iters < 1 || cg_iters > 10000 ||
+      refit_rounds < 0 || refit_rounds > 100 || !(rho_rel > 0.f) || rho_rel > 1e30f)
+    return OB_ERR_UNSUPPORTED;
+  if (!W || !omega || !SA_packed || !SB_packed || !a || !m || !b || !workspace) return OB_ERR_NULL;
+  if (misaligned(W) || misaligned(omega) || misaligned(SA_packed) || misaligned(SB_packed) || misaligned(a) ||
+      misaligned(m) || misaligned(b) || misaligned(workspace))
+    return OB_ERR_ALIGN;
+  if (ws_bytes < dbf_factorize_workspace_bytes(N, K, r)) return OB_ERR_WORKSPACE;
+  LaunchCtx c;
+  ob_status st = make_ctx(stream, &c);
+  if (st != OB_OK) return st;
+  return run_dbf_factorize(W, N, K, r, omega, sweeps, admm_iters, cg_iters, rho_rel, refit_rounds, SA_packed,
+                           SB_packed, a, m, b, history, best, error, workspace, c);
 }
 
 ob_status ob_selftest_timeout(uint64_t limit_ns, void* stream) {

@@ -1,0 +1,535 @@
+// dbf_factorize.cu -- the DBF factorisation W -> (S_A, S_B, a, m, b) on the GPU.
+//
+// "Addition is almost all you need: Compressing large language models with double
+// binary factorization" (gist.science), "Optimalisatie en Training": a heuristic of
+// alternating minimisation with ADMM, the binary constraints met by an SVID-based
+// projection.  The page gives no steps; the reading implemented here is the oracle's
+// (oracle/dbf_factorize.py) with its sketch start:
+//
+//   start   A = W Ω;  B = argmin ||W - A B|| + eps ||B||, eps = 1e-6 trace(A^T A) / r;
+//           Z_A, Z_B their SVID projections, scaled duals U_A = U_B = 0.
+//   sweep   admm_iters ADMM steps on the left factor (Z_B fixed), then as many on the
+//           right factor (Z_A fixed).  One step:
+//             X <- the solution of X (G + rho I) = R,   G = F^T F,
+//                  R = op(W) F + rho (Z - U),           rho = rho_rel trace(G) / r
+//             Z <- SVID projection of X + U:  diag(u) Sign(X + U) diag(v), u v^T the
+//                  rank-1 SVID of |X + U|
+//             U <- U + X - Z
+//           The right factor is kept transposed (K x r), so both steps have this form:
+//           left op(W) = W, F = Z_B^T; right op(W) = W^T, F = Z_A.
+//   keep    the best ||W - Z_A Z_B||_F over the start and the sweeps.
+//   refit   with the signs fixed, a, then b, then m by exact least squares,
+//           refit_rounds times.
+//
+// The r x r systems are solved by conjugate gradients over the rows of X (each row is
+// one right-hand side of the symmetric positive definite G + rho I), warm-started from
+// the previous X, a fixed number of iterations; the oracle solves exactly, so the two
+// agree to the iteration's convergence.  Dense products run on a plain fp32 tiled GEMM:
+// this is offline work (a few hundred N x K x r products per weight matrix).
+#include <algorithm>
+#include <cmath>
+
+#include "ob_device.cuh"
+#include "ob_internal.h"
+
+namespace ob {
+namespace {
+
+// ------------------------------------------------------------------ fp32 GEMM
+// C (M x N, row stride ldc) = alpha * op(A) * op(B) + beta * C, all row-major.
+// op(A) is M x K: A itself (M x K, stride lda) or, with TA, the transpose of A (K x M).
+// op(B) is K x N: B itself (K x N, stride ldb) or, with TB, the transpose of B (N x K).
+// 64 x 64 tiles, k steps of 16, 256 threads with 4 x 4 outputs each.  beta == 0 never
+// reads C.
+constexpr int kTile = 64;
+constexpr int kKStep = 16;
+
+template <bool TA, bool TB>
+__global__ void __launch_bounds__(256) sgemm_kernel(int64_t M, int64_t N, int64_t K, float alpha,
+                                                    const float* __restrict__ A, int64_t lda,
+                                                    const float* __restrict__ B, int64_t ldb, float beta,
+                                                    float* __restrict__ C, int64_t ldc) {
+  __shared__ float As[kKStep][kTile + 4];
+  __shared__ float Bs[kKStep][kTile + 4];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int64_t m0 = (int64_t)blockIdx.y * kTile, n0 = (int64_t)blockIdx.x * kTile;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int64_t k0 = 0; k0 < K; k0 += kKStep) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = tid + 256 * q;  // 0 .. 1023: one element of each 64 x 16 tile
+      // Consecutive threads walk the operand's contiguous dimension.
+      const int am = TA ? (e & 63) : (e >> 4), ak = TA ? (e >> 6) : (e & 15);
+      const int64_t gm = m0 + am, gka = k0 + ak;
+      As[ak][am] = (gm < M && gka < K) ? (TA ? A[gka * lda + gm] : A[gm * lda + gka]) : 0.f;
+      const int bn = TB ? (e >> 4) : (e & 63), bk = TB ? (e & 15) : (e >> 6);
+      const int64_t gn = n0 + bn, gkb = k0 + bk;
+      Bs[bk][bn] = (gn < N && gkb < K) ? (TB ? B[gn * ldb + gkb] : B[gkb * ldb + gn]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kKStep; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t gn = n0 + tx * 4 + j;
+      if (gn >= N) continue;
+      float* c = C + gm * ldc + gn;
+      *c = beta == 0.f ? alpha * acc[i][j] : fmaf(alpha, acc[i][j], beta * *c);
+    }
+  }
+}
+
+cudaError_t gemm(bool ta, bool tb, int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
+                 const float* B, int64_t ldb, float beta, float* C, int64_t ldc, cudaStream_t s) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  const dim3 grid((unsigned)((N + kTile - 1) / kTile), (unsigned)((M + kTile - 1) / kTile));
+  if (grid.y > 65535u) return cudaErrorInvalidValue;
+  if (!ta && !tb)
+    sgemm_kernel<false, false><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc);
+  else if (ta && !tb)
+    sgemm_kernel<true, false><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc);
+  else if (!ta && tb)
+    sgemm_kernel<false, true><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc);
+  else
+    sgemm_kernel<true, true><<<grid, 256, 0, s>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ elementwise
+
+unsigned blocks_for(int64_t n) {
+  const int64_t b = (n + 255) / 256;
+  return (unsigned)(b < 4096 ? (b < 1 ? 1 : b) : 4096);
+}
+
+#define OB_GRID_STRIDE(i, n) \
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (n); i += (int64_t)gridDim.x * blockDim.x)
+
+// Z = diag(u) Sign(M) diag(v) (rows x cols); Sign(x) = -1 iff x < 0.
+__global__ void structured_kernel(const float* __restrict__ M, const float* __restrict__ u,
+                                  const float* __restrict__ v, float* __restrict__ Z, int64_t rows, int64_t cols) {
+  OB_GRID_STRIDE(i, rows * cols) {
+    const int64_t r = i / cols, c = i - r * cols;
+    const float s = M[i] < 0.f ? -1.f : 1.f;
+    Z[i] = s * u[r] * v[c];
+  }
+}
+
+// R += rho (Z - U)
+__global__ void admm_rhs_kernel(float* __restrict__ R, const float* __restrict__ Z, const float* __restrict__ U,
+                                const float* __restrict__ rho_p, int64_t n) {
+  const float rho = *rho_p;
+  OB_GRID_STRIDE(i, n) R[i] += rho * (Z[i] - U[i]);
+}
+
+// out = x + y
+__global__ void add_kernel(const float* __restrict__ x, const float* __restrict__ y, float* __restrict__ out,
+                           int64_t n) {
+  OB_GRID_STRIDE(i, n) out[i] = x[i] + y[i];
+}
+
+// U += X - Z
+__global__ void dual_kernel(float* __restrict__ U, const float* __restrict__ X, const float* __restrict__ Z,
+                            int64_t n) {
+  OB_GRID_STRIDE(i, n) U[i] += X[i] - Z[i];
+}
+
+// out = x * y (elementwise; out may be x)
+__global__ void mul_kernel(const float* x, const float* y, float* out, int64_t n) {
+  OB_GRID_STRIDE(i, n) out[i] = x[i] * y[i];
+}
+
+__global__ void fill_kernel(float* __restrict__ x, float v, int64_t n) {
+  OB_GRID_STRIDE(i, n) x[i] = v;
+}
+
+// out (cols x rows) = in (rows x cols)^T
+__global__ void transpose_kernel(const float* __restrict__ in, float* __restrict__ out, int64_t rows,
+                                 int64_t cols) {
+  OB_GRID_STRIDE(i, rows * cols) {
+    const int64_t r = i / cols, c = i - r * cols;
+    out[c * rows + r] = in[i];
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// *out = scale * trace(G) / r (G r x r), clamped at 0.  One block of 256 threads.
+__global__ void trace_scale_kernel(const float* __restrict__ G, int64_t r, float scale, float* __restrict__ out) {
+  __shared__ double part[256];
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < r; i += 256) s += (double)G[i * r + i];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double v = (double)scale * part[0] / (double)r;
+    *out = v > 0.0 ? (float)v : 0.f;
+  }
+}
+
+// *acc += sum_i (W[i] - C[i])^2 (double, one atomic per block).
+__global__ void sqdiff_kernel(const float* __restrict__ W, const float* __restrict__ C, int64_t n,
+                              double* __restrict__ acc) {
+  __shared__ double part[256];
+  double s = 0.0;
+  OB_GRID_STRIDE(i, n) {
+    const double d = (double)W[i] - (double)C[i];
+    s += d * d;
+  }
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) atomicAdd(acc, part[0]);
+}
+
+// Per row n (one warp): out[n] = <W_n, C_n> / ||C_n||^2, 0 where ||C_n|| = 0.
+__global__ void row_ratio_kernel(const float* __restrict__ W, const float* __restrict__ C, int64_t rows,
+                                 int64_t cols, float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  float num = 0.f, den = 0.f;
+  for (int64_t j = lane; j < cols; j += 32) {
+    const float c = C[row * cols + j];
+    num = fmaf(W[row * cols + j], c, num);
+    den = fmaf(c, c, den);
+  }
+  num = warp_sum(num);
+  den = warp_sum(den);
+  if (lane == 0) out[row] = den > 0.f ? num / den : 0.f;
+}
+
+// Per column k (one thread): ratio: out[k] = <X[:, k], Y[:, k]> / ||Y[:, k]||^2 (0 where
+// the norm is 0); otherwise out[k] = <X[:, k], Y[:, k]>.
+__global__ void col_dot_kernel(const float* __restrict__ X, const float* __restrict__ Y, int64_t rows,
+                               int64_t cols, bool ratio, float* __restrict__ out) {
+  OB_GRID_STRIDE(k, cols) {
+    double num = 0.0, den = 0.0;
+    for (int64_t i = 0; i < rows; ++i) {
+      const double y = Y[i * cols + k];
+      num += (double)X[i * cols + k] * y;
+      den += y * y;
+    }
+    out[k] = ratio ? (den > 0.0 ? (float)(num / den) : 0.f) : (float)num;
+  }
+}
+
+// Conjugate gradients on X (G + rho I) = R, row by row (one warp per row).
+// Start: T = X G (given); Res = R - T - rho X (in place of R), P = Res, rr = ||Res_n||^2.
+__global__ void cg_init_kernel(const float* __restrict__ X, float* __restrict__ R, const float* __restrict__ T,
+                               float* __restrict__ P, float* __restrict__ rr, const float* __restrict__ rho_p,
+                               int64_t rows, int64_t r) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float rho = *rho_p;
+  float s = 0.f;
+  for (int64_t j = lane; j < r; j += 32) {
+    const int64_t i = row * r + j;
+    const float res = R[i] - T[i] - rho * X[i];
+    R[i] = res;
+    P[i] = res;
+    s = fmaf(res, res, s);
+  }
+  s = warp_sum(s);
+  if (lane == 0) rr[row] = s;
+}
+
+// One iteration, given Q = P G: alpha = rr / <P, Q + rho P>; X += alpha P;
+// Res -= alpha (Q + rho P); beta = ||Res||^2 / rr; P = Res + beta P.  A row whose
+// curvature is not positive (or whose residual is zero) stops moving.
+__global__ void cg_step_kernel(float* __restrict__ X, float* __restrict__ Res, float* __restrict__ P,
+                               const float* __restrict__ Q, float* __restrict__ rr, const float* __restrict__ rho_p,
+                               int64_t rows, int64_t r) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float rho = *rho_p;
+  float* x = X + row * r;
+  float* res = Res + row * r;
+  float* p = P + row * r;
+  const float* q = Q + row * r;
+  float pq = 0.f;
+  for (int64_t j = lane; j < r; j += 32) pq = fmaf(p[j], q[j] + rho * p[j], pq);
+  pq = warp_sum(pq);
+  const float rr0 = rr[row];
+  const float alpha = (pq > 0.f && rr0 > 0.f && isfinite(pq)) ? rr0 / pq : 0.f;
+  float rn = 0.f;
+  for (int64_t j = lane; j < r; j += 32) {
+    const float pj = p[j];
+    x[j] = fmaf(alpha, pj, x[j]);
+    const float nr = res[j] - alpha * (q[j] + rho * pj);
+    res[j] = nr;
+    rn = fmaf(nr, nr, rn);
+  }
+  rn = warp_sum(rn);
+  const float beta = (alpha != 0.f && rr0 > 0.f) ? rn / rr0 : 0.f;
+  for (int64_t j = lane; j < r; j += 32) p[j] = res[j] + beta * p[j];
+  if (lane == 0) rr[row] = alpha != 0.f ? rn : 0.f;
+}
+
+// ------------------------------------------------------------------ workspace
+
+size_t al(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct FactLayout {
+  size_t XA, ZA, UA, MA, MAb, XB, ZB, UB, MB, MBb, R, P, Q, G, G2, C;
+  size_t uA, vA, uAb, vAb, uB, vB, uBb, vBb, ones, rr, h, rho, zero, acc, svid, total;
+  FactLayout(int64_t N, int64_t K, int64_t r) {
+    const size_t f = sizeof(float);
+    const size_t L = (size_t)(N > K ? N : K);
+    const size_t V = (size_t)(L > (size_t)r ? L : (size_t)r);
+    size_t o = 0;
+    auto take = [&o](size_t bytes) {
+      const size_t at = o;
+      o = al(o + bytes);
+      return at;
+    };
+    XA = take(f * N * r); ZA = take(f * N * r); UA = take(f * N * r); MA = take(f * N * r); MAb = take(f * N * r);
+    XB = take(f * K * r); ZB = take(f * K * r); UB = take(f * K * r); MB = take(f * K * r); MBb = take(f * K * r);
+    R = take(f * L * r); P = take(f * L * r); Q = take(f * L * r);
+    G = take(f * r * r); G2 = take(f * r * r);
+    C = take(f * N * K);
+    uA = take(f * N); vA = take(f * r); uAb = take(f * N); vAb = take(f * r);
+    uB = take(f * K); vB = take(f * r); uBb = take(f * K); vBb = take(f * r);
+    ones = take(f * V); rr = take(f * L); h = take(f * r);
+    rho = take(f); zero = take(f); acc = take(sizeof(double));
+    svid = take(svid_workspace_bytes((int64_t)L, r));
+    total = o;
+  }
+};
+
+struct Ctx {
+  cudaStream_t s;
+  const LaunchCtx* lc;
+};
+
+#define OB_TRY_CUDA(x)                      \
+  do {                                      \
+    if ((x) != cudaSuccess) return OB_ERR_CUDA; \
+  } while (0)
+#define OB_TRY(x)                \
+  do {                           \
+    const ob_status st_ = (x);   \
+    if (st_ != OB_OK) return st_; \
+  } while (0)
+
+ob_status launched() { return cudaGetLastError() == cudaSuccess ? OB_OK : OB_ERR_CUDA; }
+
+// X (rows x r) <- CG solution of X (G + rho I) = R, warm-started from X.  R is overwritten
+// (the residual); P, Q (rows x r) and rr (rows) are scratch.
+ob_status cg_solve(float* X, float* R, const float* G, const float* rho, int64_t rows, int64_t r, int iters,
+                   float* P, float* Q, float* rr, cudaStream_t s) {
+  const unsigned rb = (unsigned)((rows + 7) / 8);  // 8 warps per block, one row each
+  OB_TRY_CUDA(gemm(false, false, rows, r, r, 1.f, X, r, G, r, 0.f, Q, r, s));
+  cg_init_kernel<<<rb, 256, 0, s>>>(X, R, Q, P, rr, rho, rows, r);
+  OB_TRY(launched());
+  for (int t = 0; t < iters; ++t) {
+    OB_TRY_CUDA(gemm(false, false, rows, r, r, 1.f, P, r, G, r, 0.f, Q, r, s));
+    cg_step_kernel<<<rb, 256, 0, s>>>(X, R, P, Q, rr, rho, rows, r);
+    OB_TRY(launched());
+  }
+  return OB_OK;
+}
+
+// Z = diag(u) Sign(M) diag(v) with (u, v) the rank-1 SVID of |M| (rows x r).  A power
+// iteration that reaches its cap keeps its last iterate, as the SVID entry point does.
+ob_status project(const float* M, int64_t rows, int64_t r, float* u, float* v, float* Z, void* svid_ws,
+                  const LaunchCtx& lc) {
+  const ob_status st = run_svid(M, rows, r, u, v, nullptr, 200, 1e-6f, nullptr, svid_ws, lc);
+  if (st != OB_OK && st != OB_ERR_NOT_CONVERGED) return st;
+  structured_kernel<<<blocks_for(rows * r), 256, 0, lc.stream>>>(M, u, v, Z, rows, r);
+  return launched();
+}
+
+// ||W - Z_A Z_Bt^T||_F (host value; synchronises).  C: N x K scratch.
+ob_status frob_error(const float* W, const float* ZA, const float* ZBt, int64_t N, int64_t K, int64_t r, float* C,
+                     double* acc, cudaStream_t s, double* out) {
+  OB_TRY_CUDA(gemm(false, true, N, K, r, 1.f, ZA, r, ZBt, r, 0.f, C, K, s));
+  OB_TRY_CUDA(cudaMemsetAsync(acc, 0, sizeof(double), s));
+  sqdiff_kernel<<<blocks_for(N * K), 256, 0, s>>>(W, C, N * K, acc);
+  OB_TRY(launched());
+  double h = 0.0;
+  OB_TRY_CUDA(cudaMemcpyAsync(&h, acc, sizeof(double), cudaMemcpyDeviceToHost, s));
+  OB_TRY_CUDA(cudaStreamSynchronize(s));
+  if (!std::isfinite(h)) return OB_ERR_NAN;
+  *out = std::sqrt(h);
+  return OB_OK;
+}
+
+}  // namespace
+
+size_t dbf_factorize_workspace_bytes(int64_t N, int64_t K, int64_t r) { return FactLayout(N, K, r).total; }
+
+ob_status run_dbf_factorize(const float* W, int64_t N, int64_t K, int64_t r, const float* omega, int sweeps,
+                            int admm_iters, int cg_iters, float rho_rel, int refit_rounds, uint32_t* SA_packed,
+                            uint32_t* SB_packed, float* a, float* m, float* b, float* history, float* best_out,
+                            float* error_out, void* workspace, const LaunchCtx& lc) {
+  const FactLayout Lo(N, K, r);
+  char* base = static_cast<char*>(workspace);
+  auto F = [base](size_t off) { return reinterpret_cast<float*>(base + off); };
+  float *XA = F(Lo.XA), *ZA = F(Lo.ZA), *UA = F(Lo.UA), *MA = F(Lo.MA), *MAb = F(Lo.MAb);
+  float *XB = F(Lo.XB), *ZB = F(Lo.ZB), *UB = F(Lo.UB), *MB = F(Lo.MB), *MBb = F(Lo.MBb);
+  float *R = F(Lo.R), *P = F(Lo.P), *Q = F(Lo.Q), *G = F(Lo.G), *G2 = F(Lo.G2), *C = F(Lo.C);
+  float *uA = F(Lo.uA), *vA = F(Lo.vA), *uAb = F(Lo.uAb), *vAb = F(Lo.vAb);
+  float *uB = F(Lo.uB), *vB = F(Lo.vB), *uBb = F(Lo.uBb), *vBb = F(Lo.vBb);
+  float *ones = F(Lo.ones), *rr = F(Lo.rr), *h = F(Lo.h), *rho = F(Lo.rho), *zero = F(Lo.zero);
+  double* acc = reinterpret_cast<double*>(base + Lo.acc);
+  void* svid_ws = base + Lo.svid;
+  const cudaStream_t s = lc.stream;
+  const int64_t V = std::max<int64_t>(std::max<int64_t>(N, K), r);
+
+  fill_kernel<<<blocks_for(V), 256, 0, s>>>(ones, 1.f, V);
+  fill_kernel<<<1, 32, 0, s>>>(zero, 0.f, 1);
+  OB_TRY(launched());
+
+  // ---- start: A = W Ω; B^T (K x r) solves B^T (A^T A + eps I) = W^T A.
+  OB_TRY_CUDA(gemm(false, false, N, r, K, 1.f, W, K, omega, r, 0.f, XA, r, s));
+  OB_TRY_CUDA(gemm(true, false, r, r, N, 1.f, XA, r, XA, r, 0.f, G, r, s));
+  trace_scale_kernel<<<1, 256, 0, s>>>(G, r, 1e-6f, rho);
+  OB_TRY(launched());
+  OB_TRY_CUDA(gemm(true, false, K, r, N, 1.f, W, K, XA, r, 0.f, R, r, s));
+  OB_TRY_CUDA(cudaMemsetAsync(XB, 0, sizeof(float) * K * r, s));
+  OB_TRY(cg_solve(XB, R, G, rho, K, r, 4 * cg_iters, P, Q, rr, s));
+  OB_TRY_CUDA(cudaMemcpyAsync(MA, XA, sizeof(float) * N * r, cudaMemcpyDeviceToDevice, s));
+  OB_TRY_CUDA(cudaMemcpyAsync(MB, XB, sizeof(float) * K * r, cudaMemcpyDeviceToDevice, s));
+  OB_TRY(project(MA, N, r, uA, vA, ZA, svid_ws, lc));
+  OB_TRY(project(MB, K, r, uB, vB, ZB, svid_ws, lc));
+  OB_TRY_CUDA(cudaMemsetAsync(UA, 0, sizeof(float) * N * r, s));
+  OB_TRY_CUDA(cudaMemsetAsync(UB, 0, sizeof(float) * K * r, s));
+
+  auto keep_best = [&]() -> ob_status {
+    OB_TRY_CUDA(cudaMemcpyAsync(MAb, MA, sizeof(float) * N * r, cudaMemcpyDeviceToDevice, s));
+    OB_TRY_CUDA(cudaMemcpyAsync(MBb, MB, sizeof(float) * K * r, cudaMemcpyDeviceToDevice, s));
+    OB_TRY_CUDA(cudaMemcpyAsync(uAb, uA, sizeof(float) * N, cudaMemcpyDeviceToDevice, s));
+    OB_TRY_CUDA(cudaMemcpyAsync(vAb, vA, sizeof(float) * r, cudaMemcpyDeviceToDevice, s));
+    OB_TRY_CUDA(cudaMemcpyAsync(uBb, uB, sizeof(float) * K, cudaMemcpyDeviceToDevice, s));
+    OB_TRY_CUDA(cudaMemcpyAsync(vBb, vB, sizeof(float) * r, cudaMemcpyDeviceToDevice, s));
+    return OB_OK;
+  };
+  double best = 0.0;
+  OB_TRY(frob_error(W, ZA, ZB, N, K, r, C, acc, s, &best));
+  OB_TRY(keep_best());
+
+  // ---- sweeps.  step(): one ADMM step on the factor X (rows x r) with the other factor F
+  // (frows x r) fixed; op(W) F is W F (left: F = Z_B^T, K x r) or W^T F (right: F = Z_A).
+  auto step = [&](bool left, float* X, float* Z, float* U, float* Mx, float* u, float* v, const float* Fo,
+                  int64_t rows, int64_t frows) -> ob_status {
+    OB_TRY_CUDA(gemm(true, false, r, r, frows, 1.f, Fo, r, Fo, r, 0.f, G, r, s));
+    trace_scale_kernel<<<1, 256, 0, s>>>(G, r, rho_rel, rho);
+    OB_TRY(launched());
+    if (left)
+      OB_TRY_CUDA(gemm(false, false, N, r, K, 1.f, W, K, Fo, r, 0.f, R, r, s));
+    else
+      OB_TRY_CUDA(gemm(true, false, K, r, N, 1.f, W, K, Fo, r, 0.f, R, r, s));
+    admm_rhs_kernel<<<blocks_for(rows * r), 256, 0, s>>>(R, Z, U, rho, rows * r);
+    OB_TRY(launched());
+    OB_TRY(cg_solve(X, R, G, rho, rows, r, cg_iters, P, Q, rr, s));
+    add_kernel<<<blocks_for(rows * r), 256, 0, s>>>(X, U, Mx, rows * r);
+    OB_TRY(launched());
+    OB_TRY(project(Mx, rows, r, u, v, Z, svid_ws, lc));
+    dual_kernel<<<blocks_for(rows * r), 256, 0, s>>>(U, X, Z, rows * r);
+    return launched();
+  };
+  for (int sw = 0; sw < sweeps; ++sw) {
+    for (int t = 0; t < admm_iters; ++t) OB_TRY(step(true, XA, ZA, UA, MA, uA, vA, ZB, N, K));
+    for (int t = 0; t < admm_iters; ++t) OB_TRY(step(false, XB, ZB, UB, MB, uB, vB, ZA, K, N));
+    double e = 0.0;
+    OB_TRY(frob_error(W, ZA, ZB, N, K, r, C, acc, s, &e));
+    if (history) history[sw] = (float)e;
+    if (e < best) {
+      best = e;
+      OB_TRY(keep_best());
+    }
+  }
+  if (best_out) *best_out = (float)best;
+
+  // ---- the kept iterate: a = u_A, m = v_A ⊙ v_B (v_B is Z_B's row scale: Z_B^T = diag(u_B) S_B^T diag(v_B)),
+  // b = u_B; then the least-squares refits.  Dense forms built from the kept signs:
+  //   Lm = S_A diag(m), Rb = (S_B diag(b))^T = diag(b) S_B^T, La = diag(a) S_A diag(m), Sb = S_B^T.
+  OB_TRY_CUDA(cudaMemcpyAsync(a, uAb, sizeof(float) * N, cudaMemcpyDeviceToDevice, s));
+  OB_TRY_CUDA(cudaMemcpyAsync(b, uBb, sizeof(float) * K, cudaMemcpyDeviceToDevice, s));
+  mul_kernel<<<blocks_for(r), 256, 0, s>>>(vAb, vBb, m, r);
+  OB_TRY(launched());
+  float* Lx = XA;  // N x r scratch (the iterates are no longer needed)
+  float* Rx = XB;  // K x r scratch
+  for (int t = 0; t < refit_rounds; ++t) {
+    // a: rows of R = Lm Rb^T against W.
+    structured_kernel<<<blocks_for(N * r), 256, 0, s>>>(MAb, ones, m, Lx, N, r);
+    structured_kernel<<<blocks_for(K * r), 256, 0, s>>>(MBb, b, ones, Rx, K, r);
+    OB_TRY(launched());
+    OB_TRY_CUDA(gemm(false, true, N, K, r, 1.f, Lx, r, Rx, r, 0.f, C, K, s));
+    row_ratio_kernel<<<(unsigned)((N + 7) / 8), 256, 0, s>>>(W, C, N, K, a);
+    OB_TRY(launched());
+    // b: columns of C = La Sb^T against W.
+    structured_kernel<<<blocks_for(N * r), 256, 0, s>>>(MAb, a, m, Lx, N, r);
+    structured_kernel<<<blocks_for(K * r), 256, 0, s>>>(MBb, ones, ones, Rx, K, r);
+    OB_TRY(launched());
+    OB_TRY_CUDA(gemm(false, true, N, K, r, 1.f, Lx, r, Rx, r, 0.f, C, K, s));
+    col_dot_kernel<<<blocks_for(K), 256, 0, s>>>(W, C, N, K, true, b);
+    OB_TRY(launched());
+    // m: (P^T P ∘ Q Q^T) m = h, P = diag(a) S_A (N x r), Qt = (S_B diag(b))^T (K x r),
+    // h_j = sum_k (W^T P)[k, j] Qt[k, j].  Solved by CG from zero (the least-squares
+    // solution of smallest norm when the system is singular).
+    structured_kernel<<<blocks_for(N * r), 256, 0, s>>>(MAb, a, ones, Lx, N, r);
+    structured_kernel<<<blocks_for(K * r), 256, 0, s>>>(MBb, b, ones, Rx, K, r);
+    OB_TRY(launched());
+    OB_TRY_CUDA(gemm(true, false, r, r, N, 1.f, Lx, r, Lx, r, 0.f, G, r, s));
+    OB_TRY_CUDA(gemm(true, false, r, r, K, 1.f, Rx, r, Rx, r, 0.f, G2, r, s));
+    mul_kernel<<<blocks_for(r * r), 256, 0, s>>>(G, G2, G, r * r);
+    OB_TRY(launched());
+    OB_TRY_CUDA(gemm(true, false, K, r, N, 1.f, W, K, Lx, r, 0.f, R, r, s));
+    col_dot_kernel<<<blocks_for(r), 256, 0, s>>>(R, Rx, K, r, false, h);
+    OB_TRY(launched());
+    OB_TRY_CUDA(cudaMemsetAsync(m, 0, sizeof(float) * r, s));
+    OB_TRY(cg_solve(m, h, G, zero, 1, r, 4 * cg_iters + (int)std::min<int64_t>(r, 256), P, Q, rr, s));
+  }
+  // Final error with the refitted scales: W_hat = La Rb^T.
+  structured_kernel<<<blocks_for(N * r), 256, 0, s>>>(MAb, a, m, Lx, N, r);
+  structured_kernel<<<blocks_for(K * r), 256, 0, s>>>(MBb, b, ones, Rx, K, r);
+  OB_TRY(launched());
+  double e = 0.0;
+  OB_TRY(frob_error(W, Lx, Rx, N, K, r, C, acc, s, &e));
+  if (error_out) *error_out = (float)e;
+
+  // ---- packed signs: S_A from the kept M_A (N x r); S_B from the kept M_B^T transposed.
+  OB_TRY_CUDA(launch_pack_signs(MAb, N, r, SA_packed, lc));
+  transpose_kernel<<<blocks_for(K * r), 256, 0, s>>>(MBb, R, K, r);  // R: r x K
+  OB_TRY(launched());
+  OB_TRY_CUDA(launch_pack_signs(R, r, K, SB_packed, lc));
+  OB_TRY_CUDA(cudaStreamSynchronize(s));
+  return OB_OK;
+}
+
+}  // namespace ob

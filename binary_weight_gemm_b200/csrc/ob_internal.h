@@ -65,6 +65,15 @@ ob_status run_svid(const float* W, int64_t N, int64_t K, float* a, float* b, flo
 
 cudaError_t launch_timeout_selftest(uint64_t limit_ns, const LaunchCtx& c);
 
+// DBF factorisation (dbf_factorize.cu): workspace bytes, and the whole run (synchronous;
+// arguments validated by the caller).  history / best_out / error_out are host pointers
+// (nullable).
+size_t dbf_factorize_workspace_bytes(int64_t N, int64_t K, int64_t r);
+ob_status run_dbf_factorize(const float* W, int64_t N, int64_t K, int64_t r, const float* omega, int sweeps,
+                            int admm_iters, int cg_iters, float rho_rel, int refit_rounds, uint32_t* SA_packed,
+                            uint32_t* SB_packed, float* a, float* m, float* b, float* history, float* best_out,
+                            float* error_out, void* workspace, const LaunchCtx& lc);
+
 // One layer of a persistent layer-stack launch (linear_stack.cu).
 struct StackLayerHost {
   const void* X;        // bf16 [M, K]

@@ -193,6 +193,43 @@ def dbf_linear(X: torch.Tensor, SB_packed: torch.Tensor, m: torch.Tensor, SA_pac
     return out
 
 
+def dbf_factorize_workspace_size(N: int, K: int, r: int) -> int:
+    return int(_lib.lib().dbf_factorize_workspace_size(N, K, r))
+
+
+def dbf_factorize(W: torch.Tensor, r: int, omega: torch.Tensor, sweeps: int = 20, admm_iters: int = 3,
+                  cg_iters: int = 25, rho_rel: float = 1.0, refit_rounds: int = 2,
+                  workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """DBF factorisation W ≈ diag(a) S_A diag(m) S_B diag(b) (synchronous).
+
+    W fp32 [N, K]; omega fp32 [K, r] (the start's random matrix).  Returns a dict with
+    SA_packed int32 [N, r/32], SB_packed int32 [r, K/32], a [N], m [r], b [K] (fp32, on
+    W's device), "history" (list of sweeps floats), "best" and "error" (floats).
+    """
+    N, K = W.shape
+    _need(W, "W", torch.float32)
+    _need(omega, "omega", torch.float32, (K, r))
+    dev = W.device
+    SA = torch.empty((N, r // 32), dtype=torch.int32, device=dev)
+    SB = torch.empty((r, K // 32), dtype=torch.int32, device=dev)
+    a = torch.empty(N, dtype=torch.float32, device=dev)
+    m = torch.empty(r, dtype=torch.float32, device=dev)
+    b = torch.empty(K, dtype=torch.float32, device=dev)
+    ws_bytes = dbf_factorize_workspace_size(N, K, r)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    hist = (ctypes.c_float * max(sweeps, 1))()
+    best, err = ctypes.c_float(0.0), ctypes.c_float(0.0)
+    st = _lib.lib().dbf_factorize(_ptr(W), N, K, r, _ptr(omega), int(sweeps), int(admm_iters), int(cg_iters),
+                                  float(rho_rel), int(refit_rounds), _ptr(SA), _ptr(SB), _ptr(a), _ptr(m), _ptr(b),
+                                  ctypes.cast(hist, ctypes.c_void_p), ctypes.cast(ctypes.pointer(best), ctypes.c_void_p),
+                                  ctypes.cast(ctypes.pointer(err), ctypes.c_void_p), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
+    _lib.check("dbf_factorize", st)
+    return {"SA_packed": SA, "SB_packed": SB, "a": a, "m": m, "b": b, "history": list(hist)[:sweeps],
+            "best": best.value, "error": err.value}
+
+
 def ob_selftest_timeout(limit_ns: int = 2_000_000, stream=None) -> int:
     """Run the bounded-wait self-test; returns the ob_status it reports (8 = timeout recorded)."""
     return int(_lib.lib().ob_selftest_timeout(int(limit_ns), _stream(stream)))

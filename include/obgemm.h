@@ -271,6 +271,53 @@ OB_API ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K,
                         void* Y, int y_dtype,
                         void* workspace, size_t ws_bytes, int path, void* stream);
 
+/*
+ * Bytes of device workspace dbf_factorize needs for W N x K and middle dimension r
+ * (0 for shapes it rejects).  About 4 bytes x (5 N r + 5 K r + 3 max(N, K) r + 2 r^2
+ * + N K).
+ */
+OB_API size_t dbf_factorize_workspace_size(int64_t N, int64_t K, int64_t r);
+
+/*
+ * DBF factorisation W ≈ diag(a) · S_A · diag(m) · S_B · diag(b) ("Addition is almost
+ * all you need: Compressing large language models with double binary factorization",
+ * gist.science, "Optimalisatie en Training": alternating minimisation with ADMM, the
+ * binary constraints met by an SVID-based projection; the page gives no steps).  The
+ * steps taken:
+ *   start  A = W Ω; B = the ridge least-squares fit of W ≈ A B (ridge 1e-6 trace(AᵀA)/r);
+ *          each factor projected onto {diag(u) · Sign · diag(v)} by the rank-1 SVID of
+ *          its magnitudes (OneBit's construction).
+ *   sweep  admm_iters ADMM steps on S_A's factor, then as many on S_B's: a ridge
+ *          least-squares step toward the projection (penalty rho = rho_rel · trace of
+ *          the other factor's Gram matrix / r; solved by cg_iters conjugate-gradient
+ *          iterations per row, warm-started), the projection, the dual update.
+ *   keep   the best ||W − Z_A Z_B||_F over the start and the sweeps;
+ *   refit  a, then b, then m by exact least squares with the signs fixed,
+ *          refit_rounds times.
+ * Unweighted: the page's importance weights need calibration data.
+ *   W          device fp32 N x K, row-major.
+ *   omega      device fp32 K x r: the start's random matrix (drawn by the caller).
+ *   K, r       multiples of 32 (the packed word), r >= 32; N >= 1; each at most 2^22.
+ *   SA_packed  device N x r/32 words, SB_packed device r x K/32 words: the signs in
+ *              the layout of ob_pack_signs (bit = 1 <=> -1), ready for dbf_linear.
+ *   a, m, b    device fp32 [N], [r], [K] (refitted scales may be negative).
+ *   history    host fp32 [sweeps], ||W − Z_A Z_B||_F after each sweep (nullable);
+ *   best       host fp32, the kept iterate's error (nullable);
+ *   error      host fp32, the error after the refit (nullable).
+ *   workspace  device, at least dbf_factorize_workspace_size(N, K, r) bytes.
+ * SYNCHRONOUS: returns when the result is in place (it reads the error back after
+ * every sweep).  OB_ERR_UNSUPPORTED for sweeps outside [0, 100000], admm_iters
+ * outside [1, 1000], cg_iters outside [1, 10000], refit_rounds outside [0, 100] or
+ * rho_rel not positive and finite; OB_ERR_NAN if W (or Ω) leads to a non-finite
+ * error.  Parity with the fp64 oracle is to properties, not digits: the page's
+ * method is a heuristic, and sign decisions near zero differ between precisions.
+ */
+OB_API ob_status dbf_factorize(const float* W, int64_t N, int64_t K, int64_t r, const float* omega, int sweeps,
+                               int admm_iters, int cg_iters, float rho_rel, int refit_rounds,
+                               uint32_t* SA_packed, uint32_t* SB_packed, float* a, float* m, float* b,
+                               float* history, float* best, float* error, void* workspace, size_t ws_bytes,
+                               void* stream);
+
 /* Size of the static scratch behind dbf_linear_noalloc: M * r * 2 bytes must fit. */
 #define OB_DBF_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 

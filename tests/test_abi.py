@@ -133,3 +133,38 @@ def test_layernorm_and_stack_argument_checks_without_gpu(lib):
     # a null input scale is allowed (no scale); the next check that fails is the device context
     st = lib.ob_linear_stack(layers(ObLayer(p, p, p, None, p, 64, 32, 0, 0)), 1, 4, ws, wsn, None)
     assert st not in (NULL, SHAPE, ALIGN, WS, UNSUP)
+
+
+def test_factorize_argument_checks_without_gpu(lib):
+    NULL, SHAPE, ALIGN, WS, UNSUP = 1, 2, 3, 6, 9
+    p = ctypes.c_void_p(4096)
+    bad = ctypes.c_void_p(4100)
+    ws = lib.dbf_factorize_workspace_size(64, 128, 32)
+    assert ws >= 4 * (5 * 64 * 32 + 5 * 128 * 32 + 3 * 128 * 32 + 2 * 32 * 32 + 64 * 128)
+    assert lib.dbf_factorize_workspace_size(64, 100, 32) == 0   # K not a multiple of 32
+    assert lib.dbf_factorize_workspace_size(64, 128, 48) == 0   # r not a multiple of 32
+    assert lib.dbf_factorize_workspace_size(0, 128, 32) == 0
+
+    def call(W=p, N=64, K=128, r=32, omega=p, sweeps=2, admm=3, cg=25, rho=1.0, refit=2, SA=p, SB=p, a=p, m=p,
+             b=p, work=p, wsb=ws):
+        return lib.dbf_factorize(W, N, K, r, omega, sweeps, admm, cg, rho, refit, SA, SB, a, m, b, None, None, None,
+                                 work, wsb, None)
+
+    assert call(K=100) == SHAPE
+    assert call(r=48) == SHAPE
+    assert call(r=0) == SHAPE
+    assert call(N=0) == SHAPE
+    assert call(sweeps=-1) == UNSUP
+    assert call(admm=0) == UNSUP
+    assert call(cg=0) == UNSUP
+    assert call(rho=0.0) == UNSUP
+    assert call(rho=float("nan")) == UNSUP
+    assert call(refit=-1) == UNSUP
+    assert call(W=None) == NULL
+    assert call(omega=None) == NULL
+    assert call(m=None) == NULL
+    assert call(work=None) == NULL
+    assert call(SB=bad) == ALIGN
+    assert call(wsb=ws - 1) == WS
+    # valid arguments: the next check is the device context (no GPU here)
+    assert call() not in (NULL, SHAPE, ALIGN, WS, UNSUP)
