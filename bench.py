@@ -549,6 +549,69 @@ def run_prefill(args, world, rank, local):
         }
         print(json.dumps(line), flush=True)
 
+def factorize_flops(N, K, r, sweeps, admm_iters, cg_iters, refit_rounds):
+    """fp32 multiply-add work (2 flops each) of one dbf_factorize run, as its GEMMs count it."""
+    gemm = lambda m, n, k: 2 * m * n * k  # noqa: E731
+    cg = lambda rows, iters: gemm(rows, r, r) * (iters + 1)  # noqa: E731
+    start = gemm(N, r, K) + gemm(r, r, N) + gemm(K, r, N) + cg(K, 4 * cg_iters) + gemm(N, K, r)
+    step_a = gemm(r, r, K) + gemm(N, r, K) + cg(N, cg_iters)
+    step_b = gemm(r, r, N) + gemm(K, r, N) + cg(K, cg_iters)
+    sweep = admm_iters * (step_a + step_b) + gemm(N, K, r)
+    refit = 3 * gemm(N, K, r) + gemm(r, r, N) + gemm(r, r, K) + gemm(K, r, N)
+    return start + sweeps * sweep + refit_rounds * refit + gemm(N, K, r)
+
+
+def run_factorize(args, world, rank, local):
+    """DBF factorisation of one 4096 x 4096 weight at r = 2048 (the bits of OneBit), offline.
+
+    Times whole dbf_factorize calls (synchronous: the error is read back after every
+    sweep) after one untimed call with a single sweep.  Reports seconds per weight, the
+    fp32 GEMM work done per second, and the relative error of the result.
+    """
+    import torch
+    from binary_weight_gemm_b200 import build, synth
+    build.build()
+    from binary_weight_gemm_b200 import ops
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    N = K = 4096
+    r = 2048
+    sweeps, admm_iters, cg_iters, refit_rounds = 20, 3, 25, 2
+    W = torch.from_numpy(synth.weights(1, N, K)).to(dev)
+    omega = torch.from_numpy((np.random.default_rng(11).standard_normal((K, r)) / np.sqrt(K)).astype(np.float32)).to(dev)
+    ws = torch.empty(ops.dbf_factorize_workspace_size(N, K, r), dtype=torch.uint8, device=dev)
+    ops.dbf_factorize(W, r, omega, sweeps=1, workspace=ws)
+    reps = max(1, min(args.steps, 2))
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            res = ops.dbf_factorize(W, r, omega, sweeps=sweeps, admm_iters=admm_iters, cg_iters=cg_iters,
+                                    refit_rounds=refit_rounds, workspace=ws)
+        el = time.perf_counter() - t0
+    el = max_over_ranks(el * 1e3, world) * 1e-3
+    assert ops.ob_last_device_error() == 0
+    flops = factorize_flops(N, K, r, sweeps, admm_iters, cg_iters, refit_rounds)
+    nW = float(torch.linalg.vector_norm(W).item())
+    if rank == 0:
+        line = {
+            "metric": "dbf_factorize seconds per 4096x4096 weight (r=2048)", "value": el / reps, "unit": "s",
+            "n_gpus": world, "steps": reps, "warmup": 1, "ms_per_step": el / reps * 1e3,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "dbf_factorize_4096x4096_r2048", "N": N, "K": K, "r": r, "sweeps": sweeps,
+                       "admm_iters": admm_iters, "cg_iters": cg_iters, "refit_rounds": refit_rounds,
+                       "timing": "host wall clock around synchronous calls (the call reads its error back "
+                                 "after every sweep)"},
+            "gemm_tflops": flops * reps / el / 1e12,
+            "relative_error": res["error"] / nW, "relative_error_best_iterate": res["best"] / nW,
+            "history": [h / nW for h in res["history"]],
+            "gpu_launches": None, "clocks": clocks, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+
+
 STACK_SHAPES = {"q": (4096, 4096), "k": (4096, 4096), "v": (4096, 4096), "o": (4096, 4096),
                 "gate": (4096, 11008), "up": (4096, 11008), "down": (11008, 4096)}  # name: (K, N)
 
@@ -799,9 +862,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "prefill", "stack"], default="decode",
+    ap.add_argument("--workload", choices=["decode", "prefill", "stack", "factorize"], default="decode",
                     help="decode: OneBit 4096x4096 at M=1,4,16 (default); prefill: M=2048, 4096 -> 11008; "
-                         "stack: one token through 32 blocks of 7B-shaped OneBit layers at M=1 and 16")
+                         "stack: one token through 32 blocks of 7B-shaped OneBit layers at M=1 and 16; "
+                         "factorize: DBF factorisation of a 4096x4096 weight at r=2048")
     ap.add_argument("--blocks", type=int, default=32, help="blocks of the stack workload")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-extra", dest="extra", action="store_false")
@@ -817,6 +881,8 @@ def main():
             run_prefill(args, world, rank, local)
         elif args.workload == "stack":
             run_stack(args, world, rank, local)
+        elif args.workload == "factorize":
+            run_factorize(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
