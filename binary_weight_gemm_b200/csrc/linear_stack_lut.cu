@@ -34,7 +34,6 @@
 // re-reads); the largest stall is the CTA barrier (one per 1024-k chunk, load imbalance
 // between warps when a CTA holds few rows, and the grid barrier).
 #include <algorithm>
-#include <cstring>
 
 #include <cuda_bf16.h>
 
