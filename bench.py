@@ -576,7 +576,7 @@ def run_factorize(args, world, rank, local):
     torch.cuda.set_device(dev)
     N = K = 4096
     r = 2048
-    sweeps, admm_iters, cg_iters, refit_rounds = 20, 3, 25, 2
+    sweeps, admm_iters, cg_iters, refit_rounds = 20, 3, 5, 2
     W = torch.from_numpy(synth.weights(1, N, K)).to(dev)
     omega = torch.from_numpy((np.random.default_rng(11).standard_normal((K, r)) / np.sqrt(K)).astype(np.float32)).to(dev)
     ws = torch.empty(ops.dbf_factorize_workspace_size(N, K, r), dtype=torch.uint8, device=dev)

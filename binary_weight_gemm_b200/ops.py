@@ -198,7 +198,7 @@ def dbf_factorize_workspace_size(N: int, K: int, r: int) -> int:
 
 
 def dbf_factorize(W: torch.Tensor, r: int, omega: torch.Tensor, sweeps: int = 20, admm_iters: int = 3,
-                  cg_iters: int = 25, rho_rel: float = 1.0, refit_rounds: int = 2,
+                  cg_iters: int = 5, rho_rel: float = 1.0, refit_rounds: int = 2,
                   workspace: torch.Tensor | None = None, stream=None) -> dict:
     """DBF factorisation W ≈ diag(a) S_A diag(m) S_B diag(b) (synchronous).
 

@@ -290,7 +290,8 @@ OB_API size_t dbf_factorize_workspace_size(int64_t N, int64_t K, int64_t r);
  *   sweep  admm_iters ADMM steps on S_A's factor, then as many on S_B's: a ridge
  *          least-squares step toward the projection (penalty rho = rho_rel · trace of
  *          the other factor's Gram matrix / r; solved by cg_iters conjugate-gradient
- *          iterations per row, warm-started), the projection, the dual update.
+ *          iterations per row, warm-started: 5 reach the quality of exact solves on the
+ *          cases measured), the projection, the dual update.
  *   keep   the best ||W − Z_A Z_B||_F over the start and the sweeps;
  *   refit  a, then b, then m by exact least squares with the signs fixed,
  *          refit_rounds times.
