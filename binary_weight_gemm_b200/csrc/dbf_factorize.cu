@@ -6,7 +6,9 @@
 // projection.  The page gives no steps; the reading implemented here is the oracle's
 // (oracle/dbf_factorize.py) with its sketch start:
 //
-//   start   A = W Ω;  B = argmin ||W - A B|| + eps ||B||, eps = 1e-6 trace(A^T A) / r;
+//   start   A = W Ω;  B = argmin ||W - A B||^2 + eps ||B||^2, eps = 0.1 trace(A^T A) / r
+//           (a ridge far above fp32 rounding of A^T A, so a rank-deficient W Ω stays
+//           well posed);
 //           Z_A, Z_B their SVID projections, scaled duals U_A = U_B = 0.
 //   sweep   admm_iters ADMM steps on the left factor (Z_B fixed), then as many on the
 //           right factor (Z_A fixed).  One step:
@@ -41,6 +43,7 @@ namespace {
 // op(B) is K x N: B itself (K x N, stride ldb) or, with TB, the transpose of B (N x K).
 // 64 x 64 tiles, k steps of 16, 256 threads with 4 x 4 outputs each.  beta == 0 never
 // reads C.
+constexpr float kSketchRidge = 0.1f;  // the start's ridge, in units of trace(A^T A) / r
 constexpr int kTile = 64;
 constexpr int kKStep = 16;
 
@@ -417,7 +420,7 @@ ob_status run_dbf_factorize(const float* W, int64_t N, int64_t K, int64_t r, con
   // ---- start: A = W Ω; B^T (K x r) solves B^T (A^T A + eps I) = W^T A.
   OB_TRY_CUDA(gemm(false, false, N, r, K, 1.f, W, K, omega, r, 0.f, XA, r, s));
   OB_TRY_CUDA(gemm(true, false, r, r, N, 1.f, XA, r, XA, r, 0.f, G, r, s));
-  trace_scale_kernel<<<1, 256, 0, s>>>(G, r, 1e-6f, rho);
+  trace_scale_kernel<<<1, 256, 0, s>>>(G, r, kSketchRidge, rho);
   OB_TRY(launched());
   OB_TRY_CUDA(gemm(true, false, K, r, N, 1.f, W, K, XA, r, 0.f, R, r, s));
   OB_TRY_CUDA(cudaMemsetAsync(XB, 0, sizeof(float) * K * r, s));

@@ -284,7 +284,7 @@ OB_API size_t dbf_factorize_workspace_size(int64_t N, int64_t K, int64_t r);
  * gist.science, "Optimalisatie en Training": alternating minimisation with ADMM, the
  * binary constraints met by an SVID-based projection; the page gives no steps).  The
  * steps taken:
- *   start  A = W Ω; B = the ridge least-squares fit of W ≈ A B (ridge 1e-6 trace(AᵀA)/r);
+ *   start  A = W Ω; B = the ridge least-squares fit of W ≈ A B (ridge 0.1 trace(AᵀA)/r);
  *          each factor projected onto {diag(u) · Sign · diag(v)} by the rank-1 SVID of
  *          its magnitudes (OneBit's construction).
  *   sweep  admm_iters ADMM steps on S_A's factor, then as many on S_B's: a ridge

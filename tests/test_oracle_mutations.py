@@ -6,12 +6,13 @@ the largest singular triple, a flipped unpack polarity, a dropped middle or inpu
 scale, reversed columns, an unbiased variance, a missing mean subtraction; in the
 factorisation a dropped ADMM penalty or pull, a wrong dual sign, dropped signs in
 the projection, half of the middle scale lost, a matrix instead of a Hadamard
-product in the Gram matrix, a biased refit), executes the result as fresh
-in-memory modules (nothing is written to disk) and runs a compact set of the pins
-against it: the hand-worked fixtures under tests/golden/, the pack/unpack round
-trip, Proposition 2's closed form, the DBF chain against the direct form, the
-projection's closed-form error, the ADMM steps and scale refits against library
-least squares, exact recovery of a rank-1 DBF weight and the low-rank property.
+product in the Gram matrix, a biased refit, a mis-scaled start ridge), executes
+the result as fresh in-memory modules (nothing is written to disk) and runs a
+compact set of the pins against it: the hand-worked fixtures under tests/golden/,
+the pack/unpack round trip, Proposition 2's closed form, the DBF chain against the
+direct form, the projection's closed-form error, the ADMM steps and scale refits
+against library least squares, the sketch start's closed form on a rank-1 weight,
+exact recovery of a rank-1 DBF weight and the low-rank property.
 Every mutant must fail at least one pin; the unmodified oracle must pass all of
 them.
 """
@@ -164,6 +165,13 @@ def _pins(o):
         res = o.dbf_factorize(W, 1, sweeps=2, refit_rounds=0)
         return res["error"] <= 1e-10 * np.linalg.norm(W)
 
+    def sketch_start_closed_form():
+        rng = np.random.default_rng(8)
+        W = o.dbf_weight(np.sign(rng.standard_normal((6, 1))), np.sign(rng.standard_normal((1, 8))),
+                         rng.uniform(0.2, 2, 6), rng.uniform(0.5, 2, 1), rng.uniform(0.2, 2, 8))
+        A, B = o.dbf_init_sketch(W, rng.standard_normal((8, 4)))
+        return np.allclose(A @ B, W / (1 + o.SKETCH_RIDGE / 4), rtol=1e-10, atol=1e-12)
+
     def factorize_low_rank():
         rng = np.random.default_rng(0)
         N, K = 96, 128
@@ -177,6 +185,7 @@ def _pins(o):
                      ("dbf_golden", dbf_golden), ("dbf_chain", dbf_chain), ("layernorm_golden", layernorm_golden),
                      ("projection_closed_form", projection_closed_form), ("admm_step_lstsq", admm_step_lstsq),
                      ("refit_lstsq", refit_lstsq), ("factorize_exact_rank1", factorize_exact_rank1),
+                     ("sketch_start_closed_form", sketch_start_closed_form),
                      ("factorize_low_rank", factorize_low_rank)):
         check(name, fn)
     return failed
@@ -203,6 +212,7 @@ MUTATIONS = [
     ("dbf_factorize.py", "a, m, b = uA, vA * uB, vB", "a, m, b = uA, vA, vB"),                 # middle scale half lost
     ("dbf_factorize.py", "G = (P.T @ P) * (Q @ Q.T)", "G = (P.T @ P) @ (Q @ Q.T)"),             # Gram product
     ("dbf_factorize.py", "den = (C * C).sum(axis=0)", "den = (C * C).sum(axis=0) + 1.0"),      # biased b refit
+    ("dbf_factorize.py", "eps = SKETCH_RIDGE * float(np.trace(G)) / r", "eps = SKETCH_RIDGE * float(np.trace(G))"),
 ]
 
 
