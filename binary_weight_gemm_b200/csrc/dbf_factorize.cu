@@ -26,8 +26,8 @@
 // The r x r systems are solved by conjugate gradients over the rows of X (each row is
 // one right-hand side of the symmetric positive definite G + rho I), warm-started from
 // the previous X, a fixed number of iterations; the oracle solves exactly, so the two
-// agree to the iteration's convergence.  Dense products run on a plain fp32 tiled GEMM:
-// this is offline work (a few hundred N x K x r products per weight matrix).
+// agree to the iteration's convergence.  Dense products run on a register-blocked fp32
+// SIMT GEMM (offline work: a few hundred N x K x r products per weight matrix).
 #include <algorithm>
 #include <cmath>
 
@@ -37,64 +37,94 @@
 namespace ob {
 namespace {
 
+constexpr float kSketchRidge = 0.1f;  // the start's ridge, in units of trace(A^T A) / r
+
 // ------------------------------------------------------------------ fp32 GEMM
 // C (M x N, row stride ldc) = alpha * op(A) * op(B) + beta * C, all row-major.
 // op(A) is M x K: A itself (M x K, stride lda) or, with TA, the transpose of A (K x M).
 // op(B) is K x N: B itself (K x N, stride ldb) or, with TB, the transpose of B (N x K).
-// 64 x 64 tiles, k steps of 16, 256 threads with 4 x 4 outputs each.  beta == 0 never
-// reads C.
-constexpr float kSketchRidge = 0.1f;  // the start's ridge, in units of trace(A^T A) / r
-constexpr int kTile = 64;
-constexpr int kKStep = 16;
+// 128 x 128 tiles, k steps of 8 through two shared-memory buffers (the next step's
+// elements are loaded into registers while the current one is multiplied), 256 threads
+// with 8 x 8 outputs each: rows ty*4 + i and 64 + ty*4 + i, columns tx*4 + j and
+// 64 + tx*4 + j (i, j < 4), so every shared-memory read is a float4.  Rows of the tiles
+// are padded to 132 floats: the stores of a warp then fall in 32 different banks.
+// beta == 0 never reads C.
+constexpr int kTile = 128;
+constexpr int kKStep = 8;
+constexpr int kPad = kTile + 4;
 
 template <bool TA, bool TB>
 __global__ void __launch_bounds__(256) sgemm_kernel(int64_t M, int64_t N, int64_t K, float alpha,
                                                     const float* __restrict__ A, int64_t lda,
                                                     const float* __restrict__ B, int64_t ldb, float beta,
                                                     float* __restrict__ C, int64_t ldc) {
-  __shared__ float As[kKStep][kTile + 4];
-  __shared__ float Bs[kKStep][kTile + 4];
+  __shared__ __align__(16) float As[2][kKStep][kPad];
+  __shared__ __align__(16) float Bs[2][kKStep][kPad];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int64_t m0 = (int64_t)blockIdx.y * kTile, n0 = (int64_t)blockIdx.x * kTile;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int64_t k0 = 0; k0 < K; k0 += kKStep) {
+  // Element e = tid + 256 q of each 128 x 8 tile; consecutive threads walk the operand's
+  // contiguous dimension.
+  float ra[4], rb[4];
+  auto load = [&](int64_t k0) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int e = tid + 256 * q;  // 0 .. 1023: one element of each 64 x 16 tile
-      // Consecutive threads walk the operand's contiguous dimension.
-      const int am = TA ? (e & 63) : (e >> 4), ak = TA ? (e >> 6) : (e & 15);
+      const int e = tid + 256 * q;
+      const int am = TA ? (e & 127) : (e >> 3), ak = TA ? (e >> 7) : (e & 7);
       const int64_t gm = m0 + am, gka = k0 + ak;
-      As[ak][am] = (gm < M && gka < K) ? (TA ? A[gka * lda + gm] : A[gm * lda + gka]) : 0.f;
-      const int bn = TB ? (e >> 4) : (e & 63), bk = TB ? (e & 15) : (e >> 6);
+      ra[q] = (gm < M && gka < K) ? (TA ? A[gka * lda + gm] : A[gm * lda + gka]) : 0.f;
+      const int bn = TB ? (e >> 3) : (e & 127), bk = TB ? (e & 7) : (e >> 7);
       const int64_t gn = n0 + bn, gkb = k0 + bk;
-      Bs[bk][bn] = (gn < N && gkb < K) ? (TB ? B[gn * ldb + gkb] : B[gkb * ldb + gn]) : 0.f;
+      rb[q] = (gn < N && gkb < K) ? (TB ? B[gn * ldb + gkb] : B[gkb * ldb + gn]) : 0.f;
     }
-    __syncthreads();
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = tid + 256 * q;
+      const int am = TA ? (e & 127) : (e >> 3), ak = TA ? (e >> 7) : (e & 7);
+      As[buf][ak][am] = ra[q];
+      const int bn = TB ? (e >> 3) : (e & 127), bk = TB ? (e & 7) : (e >> 7);
+      Bs[buf][bk][bn] = rb[q];
+    }
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  load(0);
+  store(0);
+  __syncthreads();
+  int buf = 0;
+  for (int64_t k0 = 0; k0 < K; k0 += kKStep) {
+    const bool more = k0 + kKStep < K;
+    if (more) load(k0 + kKStep);
 #pragma unroll
     for (int kk = 0; kk < kKStep; ++kk) {
-      float a[4], b[4];
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
     }
+    // The other buffer was last read in the previous step, which every thread finished
+    // before that step's barrier.
+    if (more) store(buf ^ 1);
     __syncthreads();
+    buf ^= 1;
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t gm = m0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int64_t gm = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
     if (gm >= M) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t gn = n0 + tx * 4 + j;
+    for (int j = 0; j < 8; ++j) {
+      const int64_t gn = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
       if (gn >= N) continue;
       float* c = C + gm * ldc + gn;
       *c = beta == 0.f ? alpha * acc[i][j] : fmaf(alpha, acc[i][j], beta * *c);
