@@ -622,7 +622,7 @@ def run_factorize(args, world, rank, local):
             "gemm_tflops": flops * reps / el / 1e12,
             "relative_error": res["error"] / nW, "relative_error_best_iterate": res["best"] / nW,
             "history": [h / nW for h in res["history"]],
-            "gpu_launches": None, "clocks": clocks, "cpu_baseline": cpu,
+            "gpu_launches": None, "clocks": clocks.summary(), "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
 

@@ -1,10 +1,16 @@
 """Build libobgemm.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage: ``python -m binary_weight_gemm_b200.build [--force] [--verbose]``.
+Usage: ``python -m binary_weight_gemm_b200.build [--force] [--verbose] [--debug-bounds]``.
 Each ``csrc/*.cu`` compiles to an object under ``_build/`` (in parallel), and
 the objects link into ``binary_weight_gemm_b200/libobgemm.so`` with the CUDA
 runtime linked statically.  A source hash stored beside the library skips the
 build when nothing changed.
+
+``--debug-bounds`` (or the environment variable ``OB_DEBUG_BOUNDS=1`` when ``build()``
+is called without the argument) compiles with ``-DOB_DEBUG_BOUNDS``: kernels that
+support it check every index they form against their buffers' lengths on the device
+and record ``OB_ERR_DEVICE_BOUNDS`` instead of touching memory outside them.  It is a
+checking build for tests, slower than the default one.
 """
 from __future__ import annotations
 
@@ -40,7 +46,15 @@ def _sources() -> list[str]:
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
 
 
-def _hash_inputs() -> str:
+def _flags(debug_bounds: bool) -> list[str]:
+    return CFLAGS + (["-DOB_DEBUG_BOUNDS"] if debug_bounds else [])
+
+
+def _debug_from_env() -> bool:
+    return os.environ.get("OB_DEBUG_BOUNDS", "") not in ("", "0")
+
+
+def _hash_inputs(debug_bounds: bool) -> str:
     h = hashlib.sha256()
     files = _sources() + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC)
                                 if f.endswith((".cuh", ".h")))
@@ -49,13 +63,17 @@ def _hash_inputs() -> str:
         h.update(f.encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
-    h.update(" ".join(ARCH + CFLAGS).encode())
+    h.update(" ".join(ARCH + _flags(debug_bounds)).encode())
     return h.hexdigest()
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    """Compile and link the library if its sources changed; return its path."""
-    digest = _hash_inputs()
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False,
+          debug_bounds: bool | None = None) -> str:
+    """Compile and link the library if its sources or flags changed; return its path."""
+    if debug_bounds is None:
+        debug_bounds = _debug_from_env()
+    flags = _flags(debug_bounds)
+    digest = _hash_inputs(debug_bounds)
     if not force and os.path.exists(LIB) and os.path.exists(STAMP):
         with open(STAMP) as f:
             if f.read().strip() == digest:
@@ -65,7 +83,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
 
     def compile_one(src: str) -> tuple[str, str]:
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-        cmd = [cc, *ARCH, *CFLAGS, "-c", src, "-o", obj]
+        cmd = [cc, *ARCH, *flags, "-c", src, "-o", obj]
         if ptxas_verbose:
             cmd += ["-Xptxas", "-v"]
         p = subprocess.run(cmd, capture_output=True, text=True)
@@ -96,5 +114,7 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true", help="print register/spill/smem use per kernel")
+    ap.add_argument("--debug-bounds", action="store_true", help="device-side index checks (-DOB_DEBUG_BOUNDS)")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose, ptxas_verbose=a.ptxas_verbose))
+    print(build(force=a.force, verbose=a.verbose, ptxas_verbose=a.ptxas_verbose,
+                debug_bounds=True if a.debug_bounds else None))

@@ -121,8 +121,15 @@ ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Largest N, K or r of dbf_factorize: its GEMM grid has one row of CTAs per 64 rows.
+// Largest N, K or r of dbf_factorize: its GEMM grid has one row of CTAs per 128 rows, so
+// 2^22 rows keep grid.y at 32768, inside the 65535 limit.
 constexpr int64_t kFactorizeMaxDim = (int64_t)1 << 22;
+
+// Largest element count of any one matrix a call may describe (2^48, far past device
+// memory): shapes are checked against it by division before any product of sizes is
+// formed, so no size computation below can wrap.
+constexpr int64_t kMaxElems = (int64_t)1 << 48;
+bool elems_ok(int64_t rows, int64_t cols) { return rows == 0 || cols <= kMaxElems / rows; }
 
 }  // namespace
 }  // namespace ob
@@ -169,7 +176,7 @@ ob_status ob_last_device_error(void* stream) {
 }
 
 ob_status ob_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* W_packed, void* stream) {
-  if (N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
+  if (N < 0 || K < 0 || K % 32 != 0 || !elems_ok(N, K)) return OB_ERR_SHAPE;
   if (N == 0 || K == 0) return OB_OK;
   if (!W || !W_packed) return OB_ERR_NULL;
   if (misaligned(W) || misaligned(W_packed)) return OB_ERR_ALIGN;
@@ -180,14 +187,14 @@ ob_status ob_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* W_packed
 }
 
 size_t ob_svid_workspace_size(int64_t N, int64_t K) {
-  if (N < 0 || K < 0) return 0;
+  if (N < 0 || K < 0 || !elems_ok(N, K)) return 0;
   return svid_workspace_bytes(N, K);
 }
 
 ob_status ob_svid_rank1(const float* W, int64_t N, int64_t K, float* a, float* b, float* sigma1, int max_iters,
                         float tol, int* iters_out, void* workspace, size_t ws_bytes, void* stream) {
   if (iters_out) *iters_out = 0;
-  if (N < 0 || K < 0 || K % 4 != 0) return OB_ERR_SHAPE;
+  if (N < 0 || K < 0 || K % 4 != 0 || !elems_ok(N, K)) return OB_ERR_SHAPE;
   if (N == 0 || K == 0) return OB_OK;
   if (!W || !a || !b) return OB_ERR_NULL;
   if (misaligned(W) || misaligned(a) || misaligned(b)) return OB_ERR_ALIGN;
@@ -204,6 +211,7 @@ ob_status ob_svid_rank1(const float* W, int64_t N, int64_t K, float* a, float* b
 ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,
                        const float* b, void* Y, int y_dtype, int path, void* stream) {
   if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
+  if (!elems_ok(M, K) || !elems_ok(N, K) || !elems_ok(M, N)) return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
   if (path < OB_PATH_AUTO || path > OB_PATH_MMA_DECODE) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
@@ -249,7 +257,8 @@ ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M, void*
   std::vector<StackLayerHost> host((size_t)n_layers);
   for (int i = 0; i < n_layers; ++i) {
     const ob_layer& L = layers[i];
-    if (L.K < 32 || L.K % 32 != 0 || L.N < 1 || L.N > ((int64_t)1 << 35)) return OB_ERR_SHAPE;
+    if (L.K < 32 || L.K % 32 != 0 || L.N < 1 || L.N > ((int64_t)1 << 35) || !elems_ok(L.N, L.K))
+      return OB_ERR_SHAPE;
     if (L.y_dtype != OB_OUT_BF16 && L.y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
     if (!L.X || !L.W_packed || !L.a || !L.Y) return OB_ERR_NULL;
     if (misaligned(L.X) || misaligned(L.W_packed) || misaligned(L.a) || misaligned(L.Y) ||
@@ -278,7 +287,7 @@ int sms_for_sizing() {
 }
 
 size_t dbf_workspace_size(int64_t M, int64_t r) {
-  if (M < 0 || r < 0) return 0;
+  if (M < 0 || r < 0 || !elems_ok(M, r)) return 0;
   const int ks = dbf_split_k(M, r, sms_for_sizing());
   return dbf_t_bytes(M, r) + (ks > 1 ? align256((size_t)ks * (size_t)M * (size_t)r * 4) : 0);
 }
@@ -287,6 +296,8 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
                         const uint32_t* SA_packed, int64_t N, const float* a, const float* b, void* Y, int y_dtype,
                         void* workspace, size_t ws_bytes, int path, void* stream) {
   if (M < 0 || N < 0 || K < 0 || r < 0 || K % 32 != 0 || r % 32 != 0) return OB_ERR_SHAPE;
+  if (!elems_ok(M, K) || !elems_ok(r, K) || !elems_ok(M, r) || !elems_ok(N, r) || !elems_ok(M, N))
+    return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
   if (path < OB_PATH_AUTO || path > OB_PATH_MMA_DECODE) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
@@ -349,9 +360,10 @@ ob_status dbf_linear(const void* X, int64_t M, int64_t K, const uint32_t* SB_pac
 ob_status dbf_linear_noalloc(const void* X, int64_t M, int64_t K, const uint32_t* SB_packed, int64_t r,
                              const float* m, const uint32_t* SA_packed, int64_t N, const float* a, const float* b,
                              void* Y, int y_dtype, void* stream) {
-  // Size check first, before any CUDA call: the intermediate is M x r bf16.
+  // Size check first, before any CUDA call: the intermediate is M x r bf16.  Checked by
+  // division so that no product of the sizes can wrap.
   if (M < 0 || r < 0) return OB_ERR_SHAPE;
-  if ((size_t)M * (size_t)r * 2 > (size_t)OB_DBF_NOALLOC_SCRATCH_BYTES) return OB_ERR_WORKSPACE;
+  if (r > 0 && M > (int64_t)(OB_DBF_NOALLOC_SCRATCH_BYTES / 2) / r) return OB_ERR_WORKSPACE;
   // Device address of the static scratch on the current device, looked up once per
   // device with that device current.  The array's name in host code is only a
   // host-side handle, never a device address.

@@ -337,6 +337,11 @@ OB_API ob_status dbf_factorize(const float* W, int64_t N, int64_t K, int64_t r, 
  * another allocator that a raw cudaMalloc would bypass.  This call itself
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
  *
+ * The array holds only the intermediate, so the first product never takes the
+ * split over K that dbf_linear uses when its workspace also holds fp32 partial
+ * sums (M = 512, r = 2048 is such a case): there this call runs that product
+ * unsplit, a few microseconds slower than dbf_linear with a full workspace.
+ *
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it; make that first call before any stream
  * capture.  Returns OB_ERR_WORKSPACE, launching nothing, when M * r * 2 bytes

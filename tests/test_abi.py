@@ -168,3 +168,20 @@ def test_factorize_argument_checks_without_gpu(lib):
     assert call(wsb=ws - 1) == WS
     # valid arguments: the next check is the device context (no GPU here)
     assert call() not in (NULL, SHAPE, ALIGN, WS, UNSUP)
+
+
+def test_sizes_whose_products_wrap_are_rejected_without_gpu(lib):
+    # Shapes whose element counts overflow 64 bits when multiplied must be refused by the
+    # host checks (OB_ERR_SHAPE / OB_ERR_WORKSPACE), never reach a launch.
+    SHAPE, WS = 2, 6
+    p = ctypes.c_void_p(4096)
+    M, r = 1 << 37, 1 << 26          # M * r * 2 == 2**64: wraps to 0 in size_t
+    assert lib.dbf_linear_noalloc(p, M, 64, p, r, p, p, 4, p, p, p, 0, None) == WS
+    assert lib.dbf_linear(p, M, 64, p, r, p, p, 4, p, p, p, 0, p, 1 << 20, None) == SHAPE
+    assert lib.dbf_workspace_size(M, r) == 0
+    big = 1 << 40
+    assert lib.ob_linear(p, big, big, p, 4, p, p, p, 0, None) == SHAPE
+    assert lib.ob_linear(p, 4, big, p, big, p, p, p, 0, None) == SHAPE
+    assert lib.ob_pack_signs(p, big, big, p, None) == SHAPE
+    assert lib.ob_svid_workspace_size(big, big) == 0
+    assert lib.ob_svid_rank1(p, big, big, p, p, None, 0, 0.0, None, p, 1 << 20, None) == SHAPE

@@ -6,11 +6,8 @@ to properties, not digits: exact recovery of a weight that is itself a rank-1 DB
 the error the outputs actually give (recomputed by the oracle from the packed signs
 and the scales), a better error than OneBit at equal bits on a low-rank weight and
 closeness to the oracle's own run from the same start matrix, and the packed signs
-feeding dbf_linear.
-
-Skipped until the entry point has run on a B200 for the first time; its host-side
-argument checks are tested on the CPU in test_abi.py, and its orchestration was
-checked against a NumPy mirror of the same steps.
+feeding dbf_linear.  Every test also reads the device error word, so a build with
+OB_DEBUG_BOUNDS=1 (device-side index checks) fails here on any refused access.
 """
 import numpy as np
 import pytest
@@ -21,7 +18,7 @@ from oracle import dbf_factorize as F
 from binary_weight_gemm_b200 import synth
 from helpers import assert_gemm_close
 
-pytestmark = [pytest.mark.gpu, pytest.mark.skip(reason="dbf_factorize has not yet run on a B200")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")
