@@ -350,25 +350,32 @@ def run_ours(args, world, rank, local):
                          "tflops_equiv": 2 * m * N_DIM * K_DIM / t_call / 1e12,
                          "frac_hbm": decode_call_bytes(m) / t_call / 1e9 / peaks["hbm_gbs"]}
 
-    # The warp-level MMA kernel forced at M = 1, for comparison with the table-driven kernel AUTO picks.
-    with torch.cuda.stream(stream):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for (P, a, b) in pool:
-                ops.ob_linear(xs[1], P, a, b, out=ys[1], path=ops.OB_PATH_MMA_DECODE, stream=stream)
-        g.replay()
-        stream.synchronize()
-        reps = max(3, args.steps // 4)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
+    # Kernels forced by path, for comparison with the ones AUTO picks (same pool, same graphs).
+    def time_forced(m, path):
+        with torch.cuda.stream(stream):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for (P, a, b) in pool:
+                    ops.ob_linear(xs[m], P, a, b, out=ys[m], path=path, stream=stream)
             g.replay()
-        e1.record(stream)
-        stream.synchronize()
-    t_call = e0.elapsed_time(e1) * 1e-3 / (reps * L)
-    per_m["1_mma_forced"] = {"us_per_call": t_call * 1e6, "hbm_gbs": decode_call_bytes(1) / t_call / 1e9,
-                             "frac_hbm": decode_call_bytes(1) / t_call / 1e9 / peaks["hbm_gbs"]}
-    del g
+            stream.synchronize()
+            reps = max(3, args.steps // 4)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+            stream.synchronize()
+        del g
+        t = e0.elapsed_time(e1) * 1e-3 / (reps * L)
+        return {"us_per_call": t * 1e6, "hbm_gbs": decode_call_bytes(m) / t / 1e9,
+                "frac_hbm": decode_call_bytes(m) / t / 1e9 / peaks["hbm_gbs"]}
+
+    for name, code in (("mma", ops.OB_PATH_MMA_DECODE), ("f8", ops.OB_PATH_F8), ("lut", ops.OB_PATH_SIMT)):
+        for m in DECODE_MS:
+            if name == "lut" and m > 1:
+                continue
+            per_m[f"{m}_{name}_forced"] = time_forced(m, code)
 
     # Dominant kernel of the step: the warp-level MMA decode kernel, which serves the M = 4 and
     # M = 16 calls (one launch each); its achieved bandwidth is its algorithmic bytes over its own
@@ -720,22 +727,13 @@ def run_stack(args, world, rank, local):
             pgraphs[m] = torch.cuda.CUDAGraph()
             with torch.cuda.graph(pgraphs[m], stream=stream):
                 ops.ob_linear_stack(specs[m], m, workspace=ws, stream=stream)
-        # The table-lookup stack kernel (OB_STACK_LUT=1, one token) is timed beside the
-        # default warp-MMA form.
+        # The bf16 warp-MMA stack form forced at one token, beside the fp8 form AUTO takes.
         mgraphs = {}
-        old = os.environ.get("OB_STACK_LUT")
-        os.environ["OB_STACK_LUT"] = "1"
-        try:
-            ops.ob_linear_stack(specs[1], 1, workspace=ws, stream=stream)
-            stream.synchronize()
-            mgraphs[1] = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(mgraphs[1], stream=stream):
-                ops.ob_linear_stack(specs[1], 1, workspace=ws, stream=stream)
-        finally:
-            if old is None:
-                del os.environ["OB_STACK_LUT"]
-            else:
-                os.environ["OB_STACK_LUT"] = old
+        ops.ob_linear_stack(specs[1], 1, workspace=ws, stream=stream, path=ops.OB_PATH_MMA_DECODE)
+        stream.synchronize()
+        mgraphs[1] = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(mgraphs[1], stream=stream):
+            ops.ob_linear_stack(specs[1], 1, workspace=ws, stream=stream, path=ops.OB_PATH_MMA_DECODE)
     calls = 7 * blocks
 
     def step():
@@ -744,7 +742,7 @@ def run_stack(args, world, rank, local):
 
     ms_max, ms, clocks = _timed(step, args, world, stream, local)
     per_m = {}
-    for mode, gs in (("persistent", pgraphs), ("per_call", graphs), ("persistent_lut", mgraphs)):
+    for mode, gs in (("persistent", pgraphs), ("per_call", graphs), ("persistent_bf16mma", mgraphs)):
         for m in gs:
             reps = max(3, args.steps // 2)
             with torch.cuda.stream(stream):
@@ -775,8 +773,8 @@ def run_stack(args, world, rank, local):
                        "layers_per_token": calls, "weights_mb": wbytes / 1e6,
                        "l2": f"inputs larger than L2: {blocks * 7} distinct weight buffers ({wbytes / 1e6:.0f} MB)",
                        "graph": "one CUDA graph per token and M holding one ob_linear_stack (persistent, "
-                                "grid barriers between dependent layers; warp-MMA kernel, "
-                                "persistent_lut_M1 the table-lookup kernel); per_call_* times one ob_linear "
+                                "grid barriers between dependent layers; AUTO: fp8 form at M=1, bf16 warp-MMA "
+                                "form at M=16; persistent_bf16mma_M1 forces the bf16 form); per_call_* times one ob_linear "
                                 "per layer in a graph with programmatic dependent launch",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "per_m": per_m,

@@ -17,7 +17,7 @@ STATUS_NAMES = {
     9: "OB_ERR_UNSUPPORTED", 10: "OB_ERR_DEVICE_BOUNDS",
 }
 OB_OUT_BF16, OB_OUT_F32 = 0, 1
-OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC_DECODE, OB_PATH_TC, OB_PATH_MMA_DECODE = 0, 1, 2, 3, 4
+OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC, OB_PATH_MMA_DECODE, OB_PATH_F8 = 0, 1, 3, 4, 5
 
 
 
@@ -43,6 +43,7 @@ SIGNATURES = {
     "ob_linear_ln": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _F, _I, _P]),
     "ob_stack_workspace_size": (_SZ, []),
     "ob_linear_stack": (_I, [ctypes.POINTER(ObLayer), _I, _I64, _P, _SZ, _P]),
+    "ob_linear_stack_ex": (_I, [ctypes.POINTER(ObLayer), _I, _I64, _P, _SZ, _I, _P]),
     "dbf_workspace_size": (_SZ, [_I64, _I64]),
     "dbf_linear": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P, _P, _I, _P, _SZ, _P]),
     "dbf_linear_ex": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P, _P, _I, _P, _SZ, _I, _P]),

@@ -2,7 +2,6 @@
 //
 // Host-side argument checks, kernel dispatch and the per-device error word.
 // Checks run before any CUDA call, so a rejected call launches nothing.
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -53,18 +52,6 @@ ob_status current_device(DeviceInfo* out) {
   return OB_OK;
 }
 
-bool env_flag(const char* name, bool dflt) {
-  const char* s = std::getenv(name);
-  if (!s || !*s) return dflt;
-  return !(s[0] == '0' || s[0] == 'n' || s[0] == 'N' || s[0] == 'f' || s[0] == 'F');
-}
-
-int decode_max_m() {
-  const char* s = std::getenv("OB_DECODE_MAX_M");
-  int v = s ? std::atoi(s) : kDecodeMaxM;
-  return v < 0 ? 0 : v;
-}
-
 ob_status make_ctx(void* stream, LaunchCtx* c) {
   DeviceInfo d;
   ob_status st = current_device(&d);
@@ -73,8 +60,8 @@ ob_status make_ctx(void* stream, LaunchCtx* c) {
   c->stream = static_cast<cudaStream_t>(stream);
   c->err = d.err;
   c->num_sms = d.num_sms;
-  c->pdl = env_flag("OB_PDL", true);
-  c->l2_prefetch = env_flag("OB_L2_PREFETCH", true);
+  c->pdl = true;
+  c->l2_prefetch = true;
   return OB_OK;
 }
 
@@ -99,20 +86,18 @@ ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) 
   // MMA kernel, more on the tcgen05 GEMM.  K beyond the tcgen05 GEMM's limit goes
   // to the warp-level MMA kernel, 16 tokens per launch.
   if (path == OB_PATH_AUTO) {
-    path = g.M == 1 ? OB_PATH_SIMT : (g.M <= decode_max_m() ? OB_PATH_MMA_DECODE : OB_PATH_TC);
+    path = g.M == 1 ? OB_PATH_SIMT : (g.M <= kDecodeMaxM ? OB_PATH_MMA_DECODE : OB_PATH_TC);
     if (path == OB_PATH_TC && g.K > sign_gemm_tc_max_k()) path = OB_PATH_MMA_DECODE;
   }
   cudaError_t e;
   switch (path) {
     case OB_PATH_SIMT: e = launch_sign_gemm_simt(g, c); break;
-    case OB_PATH_TC_DECODE: e = launch_sign_gemm_tc_decode(g, c); break;
     case OB_PATH_MMA_DECODE: e = launch_sign_gemm_mma_decode(g, c); break;
+    case OB_PATH_F8: e = launch_sign_gemm_f8(g, c); break;
     case OB_PATH_TC:
       // The CTA-pair kernel where it applies (bf16 Y, M >= 512, R >= 256, K <= 16384):
       // 1260 vs 1170 TFLOP/s for the one-CTA kernel at the prefill workload on B200.
-      // OB_TC2=0 selects the one-CTA kernel.
-      e = (env_flag("OB_TC2", true) && sign_gemm_tc2_supported(g)) ? launch_sign_gemm_tc2(g, c)
-                                                                    : launch_sign_gemm_tc(g, c);
+      e = sign_gemm_tc2_supported(g) ? launch_sign_gemm_tc2(g, c) : launch_sign_gemm_tc(g, c);
       break;
     default: return OB_ERR_UNSUPPORTED;
   }
@@ -120,6 +105,10 @@ ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) 
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Largest M the fp8 form of the layer stack takes (its activation limbs for up to two
+// tokens fill one n8 tile).
+constexpr int64_t kStackF8MaxM = 2;
 
 // Largest N, K or r of dbf_factorize: its GEMM grid has one row of CTAs per 128 rows, so
 // 2^22 rows keep grid.y at 32768, inside the 65535 limit.
@@ -213,7 +202,7 @@ ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
   if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
   if (!elems_ok(M, K) || !elems_ok(N, K) || !elems_ok(M, N)) return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
-  if (path < OB_PATH_AUTO || path > OB_PATH_MMA_DECODE) return OB_ERR_UNSUPPORTED;
+  if (path < OB_PATH_AUTO || path > OB_PATH_F8 || path == 2) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   if (K > 0 && (!X || !W_packed || !b)) return OB_ERR_NULL;
@@ -246,9 +235,11 @@ ob_status ob_linear_ln(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
 
 size_t ob_stack_workspace_size(void) { return 256; }
 
-ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M, void* workspace, size_t ws_bytes,
-                          void* stream) {
+ob_status ob_linear_stack_ex(const ob_layer* layers, int n_layers, int64_t M, void* workspace, size_t ws_bytes,
+                             int path, void* stream) {
   if (n_layers < 0 || M < 0 || M > kDecodeMaxM) return OB_ERR_SHAPE;
+  if (path != OB_PATH_AUTO && path != OB_PATH_MMA_DECODE && path != OB_PATH_F8) return OB_ERR_UNSUPPORTED;
+  if (path == OB_PATH_F8 && M > kStackF8MaxM) return OB_ERR_UNSUPPORTED;
   if (n_layers == 0 || M == 0) return OB_OK;
   if (!layers) return OB_ERR_NULL;
   if (!workspace) return OB_ERR_NULL;
@@ -269,16 +260,25 @@ ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M, void*
   LaunchCtx c;
   ob_status st = make_ctx(stream, &c);
   if (st != OB_OK) return st;
-  return status_of(launch_sign_stack(host.data(), n_layers, M, static_cast<unsigned*>(workspace), c,
-                                     env_flag("OB_STACK_LUT", false)));
+  if (path == OB_PATH_AUTO) path = M <= kStackF8MaxM ? OB_PATH_F8 : OB_PATH_MMA_DECODE;
+  return status_of(launch_sign_stack(host.data(), n_layers, M, static_cast<unsigned*>(workspace), c, path));
+}
+
+ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  return ob_linear_stack_ex(layers, n_layers, M, workspace, ws_bytes, OB_PATH_AUTO, stream);
 }
 
 // Bytes of the bf16 intermediate T: the smallest workspace dbf_linear accepts.
 size_t dbf_t_bytes(int64_t M, int64_t r) { return align256((size_t)M * (size_t)r * 2); }
 
+// Bytes after T that hold the grid-barrier word of the one-launch decode chain; fp32
+// partial sums of a split product start after them.
+constexpr size_t kDbfBarrierBytes = 256;
+
 // K slices of DBF's first product (T = ... S_B^T, M x r) when it runs on the tcgen05 GEMM.
 int dbf_split_k(int64_t M, int64_t r, int num_sms) {
-  return M > decode_max_m() ? tc_split_k(M, r, num_sms) : 1;
+  return M > kDecodeMaxM ? tc_split_k(M, r, num_sms) : 1;
 }
 
 int sms_for_sizing() {
@@ -288,8 +288,9 @@ int sms_for_sizing() {
 
 size_t dbf_workspace_size(int64_t M, int64_t r) {
   if (M < 0 || r < 0 || !elems_ok(M, r)) return 0;
+  if (M == 0 || r == 0) return 0;  // nothing to hold
   const int ks = dbf_split_k(M, r, sms_for_sizing());
-  return dbf_t_bytes(M, r) + (ks > 1 ? align256((size_t)ks * (size_t)M * (size_t)r * 4) : 0);
+  return dbf_t_bytes(M, r) + kDbfBarrierBytes + (ks > 1 ? align256((size_t)ks * (size_t)M * (size_t)r * 4) : 0);
 }
 
 ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_packed, int64_t r, const float* m,
@@ -299,7 +300,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   if (!elems_ok(M, K) || !elems_ok(r, K) || !elems_ok(M, r) || !elems_ok(N, r) || !elems_ok(M, N))
     return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
-  if (path < OB_PATH_AUTO || path > OB_PATH_MMA_DECODE) return OB_ERR_UNSUPPORTED;
+  if (path < OB_PATH_AUTO || path > OB_PATH_F8 || path == 2) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   const bool empty_sum = (K == 0 || r == 0);
@@ -318,14 +319,24 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   if (empty_sum) return zero_output(Y, M, N, y_dtype, c.stream);
   // T = ((X ⊙ b^T) S_B^T) ⊙ m^T, rounded once to bf16, then Y = (T S_A^T) ⊙ a^T.
   uint16_t* T = static_cast<uint16_t*>(workspace);
+  const size_t t_bytes = dbf_t_bytes(M, r);
+  // Decode sizes (AUTO, M <= 16): both products in one persistent launch of the layer-stack
+  // kernels (two layers, a grid barrier between them), so T is written and read back within
+  // one kernel and stays in L2.  The barrier word sits after T in the workspace.
+  if (path == OB_PATH_AUTO && M <= kDecodeMaxM && ws_bytes >= t_bytes + kDbfBarrierBytes) {
+    const StackLayerHost two[2] = {{X, SB_packed, b, m, T, K, r, OB_OUT_BF16, 0},
+                                   {T, SA_packed, nullptr, a, Y, r, N, y_dtype, 1}};
+    unsigned* bar = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + t_bytes);
+    return status_of(
+        launch_sign_stack(two, 2, M, bar, c, M <= kStackF8MaxM ? OB_PATH_F8 : OB_PATH_MMA_DECODE));
+  }
   SignGemmArgs g1{static_cast<const uint16_t*>(X), M, K, SB_packed, r, b, m, T, r, OB_OUT_BF16};
   // Few output tiles (small M x r): split the first product over K into fp32 partial
   // sums after T in the workspace, when the workspace holds them.
-  const bool tc1 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > decode_max_m() && K <= sign_gemm_tc_max_k());
-  const bool split = env_flag("OB_DBF_SPLIT", true);  // OB_DBF_SPLIT=0: neither product is split
-  const int ks = (tc1 && split) ? dbf_split_k(M, r, c.num_sms) : 1;
-  const size_t part_off = dbf_t_bytes(M, r);
-  if (ks > 1 && path != OB_PATH_TC_DECODE && ws_bytes >= part_off + (size_t)ks * (size_t)M * (size_t)r * 4) {
+  const bool tc1 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > kDecodeMaxM && K <= sign_gemm_tc_max_k());
+  const int ks = tc1 ? dbf_split_k(M, r, c.num_sms) : 1;
+  const size_t part_off = t_bytes + kDbfBarrierBytes;
+  if (ks > 1 && ws_bytes >= part_off + (size_t)ks * (size_t)M * (size_t)r * 4) {
     g1.l2_prefetch = 0;
     st = status_of(launch_sign_gemm_tc_splitk(
         g1, ks, reinterpret_cast<float*>(static_cast<char*>(workspace) + part_off), c));
@@ -339,9 +350,9 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   // CTA-pair kernel takes it and r < 4096: measured at M = 512 on B200, r = 2048
   // unsplit on the pair kernel 42.6 us per layer against 44.7 split, r = 4704 split
   // 64.4 against 67.6 unsplit.
-  const bool tc2 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > decode_max_m() && r <= sign_gemm_tc_max_k());
-  const bool pair2 = env_flag("OB_TC2", true) && sign_gemm_tc2_supported(g2) && r < 4096;
-  const int ks2 = (tc2 && split && env_flag("OB_DBF_SPLIT2", !pair2) && M > decode_max_m())
+  const bool tc2 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > kDecodeMaxM && r <= sign_gemm_tc_max_k());
+  const bool pair2 = sign_gemm_tc2_supported(g2) && r < 4096;
+  const int ks2 = (tc2 && !pair2 && M > kDecodeMaxM)
                       ? tc_split_k(M, N, c.num_sms)
                       : 1;
   if (ks2 > 1 && ws_bytes >= part_off + (size_t)ks2 * (size_t)M * (size_t)N * 4)

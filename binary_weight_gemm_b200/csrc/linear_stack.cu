@@ -4,10 +4,9 @@
 // "proposition 1"); a decoder applies such layers one after another, a layer
 // reading the output of an earlier one.  Launched one kernel per layer, every
 // dependent layer pays a launch and a drain; here one cooperative grid walks the
-// whole list.  This file holds the warp-level MMA form (any M <= 16, the default)
-// and the launcher, which takes the table-lookup form of linear_stack_lut.cu instead
-// for one token when the caller asks for it and its shared-memory staging fits.
-// The MMA form:
+// whole list.  This file holds the bf16 warp-level MMA form (any M <= 16) and the
+// launcher, which takes the fp8 form of linear_stack_f8.cu for one or two tokens.
+// The bf16 MMA form:
 //  * A layer flagged as reading an earlier layer's output waits at a grid-wide
 //    barrier; the layers between two barriers run back to back.
 //  * A layer's rows are split into 32-row blocks dealt to the CTAs round robin,
@@ -121,7 +120,7 @@ cudaError_t launch_stack_tok(const StackParams& prm, const LaunchCtx& c) {
 int stack_max_layers_per_launch() { return kStackMaxLayers; }
 
 cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c,
-                              bool allow_lut) {
+                              int path) {
   if (n == 0 || M == 0) return cudaSuccess;
   static_assert(sizeof(StackParams) <= 32000, "kernel parameters");
   StackParams* prm = new StackParams;
@@ -142,8 +141,8 @@ cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, un
     }
     e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned), c.stream);
     if (e != cudaSuccess) break;
-    if (M == 1 && allow_lut && stack_lut_fits(*prm, c.num_sms))
-      e = launch_stack_lut(*prm, c);
+    if (path == OB_PATH_F8)
+      e = launch_stack_f8(*prm, c);
     else
       e = M == 1 ? launch_stack_tok<1>(*prm, c) : (M <= 8 ? launch_stack_tok<8>(*prm, c) : launch_stack_tok<16>(*prm, c));
   }

@@ -36,8 +36,9 @@ struct SignGemmArgs {
 cudaError_t launch_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* out, const LaunchCtx& c);
 
 cudaError_t launch_sign_gemm_simt(const SignGemmArgs& g, const LaunchCtx& c);
-cudaError_t launch_sign_gemm_tc_decode(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_mma_decode(const SignGemmArgs& g, const LaunchCtx& c);
+// fp8 tensor-core sign product for small M (linear_f8.cu, f8_block.cuh).
+cudaError_t launch_sign_gemm_f8(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c);
 // cuTensorMapEncodeTiled from the driver (null if unavailable).
 void* tensor_map_encode_tiled_fn();
@@ -86,11 +87,10 @@ struct StackLayerHost {
   int barrier;          // reads an output of an earlier layer of the list
 };
 // Runs the list (M <= 16) as cooperative launches of at most stack_max_layers_per_launch()
-// layers; bar: 8 bytes of device memory (zeroed by the launcher).  allow_lut: at M = 1,
-// use the table-lookup kernel where its staging fits (OB_STACK_LUT=1; measured slower
-// than the warp-MMA form on the 7B-shaped stack, so off by default).
+// layers; bar: 8 bytes of device memory (zeroed by the launcher).  path: OB_PATH_F8 (M <= 2)
+// for the fp8 form, OB_PATH_MMA_DECODE for the bf16 form.
 cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c,
-                              bool allow_lut);
+                              int path);
 int stack_max_layers_per_launch();
 
 // Z = LayerNorm(Y) per row of the M x N matrix Y (row stride ld elements), in place.

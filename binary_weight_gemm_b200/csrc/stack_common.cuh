@@ -1,7 +1,6 @@
 // stack_common.cuh -- the layer list and the grid-wide barrier of the persistent
-// layer-stack kernels (linear_stack.cu: warp-level MMA blocks, any M <= 16;
-// linear_stack_lut.cu: one token by table lookup with the sign rows staged in
-// shared memory).
+// layer-stack kernels (linear_stack.cu: bf16 warp-level MMA blocks, any M <= 16;
+// linear_stack_f8.cu: fp8 warp-level MMA on staged activation limbs, M <= 2).
 //
 // Each layer is  Y = [(X ⊙ b^T) W_sign^T] ⊙ a^T  ("1bit量化", blog.zerodtree.com,
 // "proposition 1").  A layer flagged `barrier` reads an output of an earlier layer
@@ -39,11 +38,8 @@ struct StackParams {
   StackLayer L[kStackMaxLayers];
 };
 
-// The one-token table-lookup stack (linear_stack_lut.cu).  stack_lut_fits says whether
-// every CTA's share of every barrier group fits its shared-memory staging buffer on a
-// grid of `grid` CTAs (and K is a multiple of 128 in every layer).
-bool stack_lut_fits(const StackParams& p, int grid);
-cudaError_t launch_stack_lut(const StackParams& p, const LaunchCtx& c);
+// The one- and two-token fp8 tensor-core stack (linear_stack_f8.cu).
+cudaError_t launch_stack_f8(const StackParams& p, const LaunchCtx& c);
 
 #ifdef __CUDACC__
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {

@@ -15,8 +15,8 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import (OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_MMA_DECODE, OB_PATH_SIMT,  # noqa: F401
-                   OB_PATH_TC, OB_PATH_TC_DECODE, ObError)
+from ._lib import (OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_F8, OB_PATH_MMA_DECODE, OB_PATH_SIMT,  # noqa: F401
+                   OB_PATH_TC, ObError)
 
 
 def _stream(stream) -> int:
@@ -132,12 +132,14 @@ def ob_stack_workspace_size() -> int:
     return int(_lib.lib().ob_stack_workspace_size())
 
 
-def ob_linear_stack(layers, M: int, workspace: torch.Tensor | None = None, stream=None) -> None:
+def ob_linear_stack(layers, M: int, workspace: torch.Tensor | None = None, stream=None,
+                    path: int = OB_PATH_AUTO) -> None:
     """Run a list of OneBit layers (M <= 16 tokens) in one persistent launch.
 
     layers: sequence of (X, W_packed, a, b, Y, after_previous); X bf16 [M, K], W_packed int32
     [N, K/32], a fp32 [N], b fp32 [K] or None, Y bf16/fp32 [M, N] (written), after_previous:
-    True if X is an output of an earlier layer of the list.
+    True if X is an output of an earlier layer of the list.  path: OB_PATH_AUTO,
+    OB_PATH_MMA_DECODE or OB_PATH_F8 (M <= 2).
     """
     arr = (_lib.ObLayer * max(1, len(layers)))()
     dev = None
@@ -155,8 +157,9 @@ def ob_linear_stack(layers, M: int, workspace: torch.Tensor | None = None, strea
         dev = X.device
     if workspace is None:
         workspace = torch.zeros(ob_stack_workspace_size(), dtype=torch.uint8, device=dev or "cuda")
-    st = _lib.lib().ob_linear_stack(arr, len(layers), M, _ptr(workspace), workspace.numel(), _stream(stream))
-    _lib.check("ob_linear_stack", st)
+    st = _lib.lib().ob_linear_stack_ex(arr, len(layers), M, _ptr(workspace), workspace.numel(), int(path),
+                                       _stream(stream))
+    _lib.check("ob_linear_stack_ex", st)
 
 
 def dbf_workspace_size(M: int, r: int) -> int:

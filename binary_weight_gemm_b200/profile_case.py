@@ -4,7 +4,7 @@
     python -m binary_weight_gemm_b200.profile_case prefill --reps 6
     python -m binary_weight_gemm_b200.profile_case dbf --m 512 --reps 6
     python -m binary_weight_gemm_b200.profile_case stack --m 1 --blocks 8 --reps 5
-    python -m binary_weight_gemm_b200.profile_case stack --m 1 --chain 128 --reps 5
+    python -m binary_weight_gemm_b200.profile_case stack --m 1 --chain 128 --reps 5 --path f8
 
 The workloads are the benchmark's: OneBit 4096 x 4096 decode at M tokens, OneBit
 prefill X 2048 x 4096 -> 11008, DBF K = N = 4096 with r = 2048, and the layer stack:
@@ -46,9 +46,12 @@ def main(argv=None) -> None:
     ap.add_argument("--reps", type=int, default=6)
     ap.add_argument("--blocks", type=int, default=8, help="stack: 7B-shaped blocks")
     ap.add_argument("--chain", type=int, default=0, help="stack: chained 1024 -> 1024 layers instead")
+    ap.add_argument("--path", choices=("auto", "mma", "f8"), default="auto",
+                    help="stack / decode: kernel form (AUTO, the bf16 warp MMA, or the fp8 form)")
     args = ap.parse_args(argv)
     dev = torch.device("cuda", 0)
     torch.cuda.init()
+    path = {"auto": ops.OB_PATH_AUTO, "mma": ops.OB_PATH_MMA_DECODE, "f8": ops.OB_PATH_F8}[args.path]
 
     if args.case in ("decode", "prefill"):
         M, N, K = (args.m or 16, 4096, 4096) if args.case == "decode" else (args.m or 2048, 11008, 4096)
@@ -65,7 +68,7 @@ def main(argv=None) -> None:
 
         def call(i):
             X, P, a, b, Y = sets[i % n_sets]
-            ops.ob_linear(X, P, a, b, out=Y)
+            ops.ob_linear(X, P, a, b, out=Y, path=path)
     elif args.case == "stack":
         M = args.m or 1
         if args.chain:
@@ -97,7 +100,7 @@ def main(argv=None) -> None:
         n_sets = 1
 
         def call(i):
-            ops.ob_linear_stack(spec, M, workspace=ws)
+            ops.ob_linear_stack(spec, M, workspace=ws, path=path)
     else:
         M, N, K, r = args.m or 512, 4096, 4096, 2048
         f = synth.dbf_factors(3, N, r, K)
@@ -125,7 +128,7 @@ def main(argv=None) -> None:
     assert ops.ob_last_device_error() == 0
     if args.case != "stack":
         desc = {"N": N, "K": K}
-    print(json.dumps({"case": args.case, "M": M, **desc, "reps": args.reps, "sets": n_sets,
+    print(json.dumps({"case": args.case, "M": M, **desc, "path": args.path, "reps": args.reps, "sets": n_sets,
                       "us_per_call": e0.elapsed_time(e1) * 1e3 / args.reps}))
 
 

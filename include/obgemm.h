@@ -80,14 +80,17 @@ typedef enum ob_out_dtype {
   OB_OUT_F32 = 1
 } ob_out_dtype;
 
-/* Kernel choice for ob_linear_ex / dbf_linear_ex. */
+/* Kernel choice for ob_linear_ex / dbf_linear_ex / ob_linear_stack_ex.  Value 2 is not used
+ * (it named a tensor-memory decode kernel that measured slower than every other path and
+ * was removed); passing it returns OB_ERR_UNSUPPORTED. */
 typedef enum ob_path {
   OB_PATH_AUTO = 0,        /* M == 1: OB_PATH_SIMT; M <= 16 or K > 32768: OB_PATH_MMA_DECODE; else OB_PATH_TC */
-  OB_PATH_SIMT = 1,        /* CUDA-core select/add mat-vec (any M; slow for M > 4) */
-  OB_PATH_TC_DECODE = 2,   /* tcgen05, signs unpacked into tensor memory, M <= 16 per pass */
+  OB_PATH_SIMT = 1,        /* CUDA-core mat-vec: one token by table lookup, more tokens by select/add */
   OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA); K <= 32768; a
                               2-CTA (cta_group::2) tile where bf16 Y, M >= 512, N >= 256, K <= 16384 */
-  OB_PATH_MMA_DECODE = 4   /* warp-level MMA, signs unpacked in registers, M <= 16 per pass */
+  OB_PATH_MMA_DECODE = 4,  /* bf16 warp-level MMA, signs unpacked in registers, M <= 16 per pass */
+  OB_PATH_F8 = 5           /* fp8 (e4m3) warp-level MMA: each packed word becomes eight operand registers
+                              with one AND each, activations in three e4m3 limbs; M <= 16 per pass */
 } ob_path;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -222,22 +225,27 @@ OB_API size_t ob_stack_workspace_size(void);
  *              concurrently running ob_linear_stack.
  * Weights and scales must not be outputs of layers of the same list.  Validation of
  * every descriptor happens before anything is launched.  Asynchronous.
- * Kernel: warp-level MMA blocks by default; with the environment variable
- * OB_STACK_LUT=1 and M == 1, a table-lookup kernel that stages each CTA's sign rows
- * in shared memory (used when every K is a multiple of 128 and every CTA's share of
- * a group fits 80 KB; otherwise the default runs).  Same results within the
- * tolerances; the default was the faster of the two on 7B-shaped layers.
+ * Kernel (OB_PATH_AUTO): M <= 2, the fp8 form (one contiguous range of 16-row tiles
+ * per CTA and barrier group, activation limbs staged once per layer per CTA, e4m3
+ * warp-level MMA); M > 2, the bf16 warp-level MMA form (32-row blocks round robin).
  */
 OB_API ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/* ob_linear_stack with an explicit form: OB_PATH_AUTO, OB_PATH_MMA_DECODE (bf16, any
+ * M <= 16) or OB_PATH_F8 (M <= 2; OB_ERR_UNSUPPORTED above).  Other values:
+ * OB_ERR_UNSUPPORTED. */
+OB_API ob_status ob_linear_stack_ex(const ob_layer* layers, int n_layers, int64_t M,
+                             void* workspace, size_t ws_bytes, int path, void* stream);
+
 /*
- * Bytes of device workspace dbf_linear uses: the M x r bf16 intermediate T and, when
- * the first product runs on the tcgen05 GEMM with fewer output tiles than half the
- * SMs of the current device (e.g. M = 512, r = 2048), fp32 partial sums for splitting
- * it over K (up to 8 x M x r x 4 bytes).  dbf_linear accepts any workspace of at least
- * the intermediate's size (M x r x 2 rounded up to 256 bytes); a smaller one than
- * this function returns runs the first product without the split.
+ * Bytes of device workspace dbf_linear uses: the M x r bf16 intermediate T, 256 bytes
+ * after it (the grid-barrier word of the one-launch decode chain) and, when the first
+ * product runs on the tcgen05 GEMM with fewer output tiles than half the SMs of the
+ * current device (e.g. M = 512, r = 2048), fp32 partial sums for splitting it over K
+ * (up to 8 x M x r x 4 bytes).  dbf_linear accepts any workspace of at least T's size
+ * (M x r x 2 rounded up to 256 bytes); a smaller one than this function returns runs the
+ * decode chain as two launches, and the first product without the split.
  */
 OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
 
@@ -254,7 +262,10 @@ OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
  *   workspace  device, at least dbf_workspace_size(M, r) bytes; holds the
  *              intermediate T = ((X ⊙ b^T) S_B^T) ⊙ m^T between the two sign
  *              products (it stays in L2 at the workload sizes).
- * K % 32 == 0, r % 32 == 0.  Asynchronous.
+ * K % 32 == 0, r % 32 == 0.  Asynchronous.  M <= 16 (decode): both products run in
+ * one persistent launch (the layer-stack kernels with a grid barrier between the two
+ * products; fp8 form for M <= 2), so T never leaves the chip's L2 between them; larger
+ * M: two tcgen05 GEMMs.
  */
 OB_API ob_status dbf_linear(const void* X, int64_t M, int64_t K,
                      const uint32_t* SB_packed, int64_t r, const float* m,

@@ -9,7 +9,7 @@ from helpers import assert_gemm_close
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc_decode": 2, "tc": 3, "mma_decode": 4, "auto": 0}
+PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "f8": 5, "auto": 0}
 
 
 @pytest.fixture(scope="module")
@@ -39,7 +39,7 @@ def _ref(x, f):
     return oracle.dbf_linear(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"])
 
 
-@pytest.mark.parametrize("path", ["simt", "tc_decode", "tc", "mma_decode"])
+@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "f8", "auto"])
 @pytest.mark.parametrize("M,N,r,K", [(1, 128, 32, 64), (4, 256, 96, 256), (7, 200, 160, 96), (33, 130, 64, 128),
                                      (260, 256, 128, 320)])
 def test_dbf_small_shapes(ops, path, M, N, r, K):
@@ -48,7 +48,7 @@ def test_dbf_small_shapes(ops, path, M, N, r, K):
     assert_gemm_close(_run(ops, xb, f, PATHS[path]), _ref(x, f), what=f"dbf {path} {M},{N},{r},{K}")
 
 
-@pytest.mark.parametrize("M", [1, 512])
+@pytest.mark.parametrize("M", [1, 2, 16, 512])
 def test_dbf_workload_full(ops, M):
     # DBF: K = N = 4096, r = 2048; S_A, S_B random +/-1; a, m, b ~ |N(0,1)|*0.02+1e-3.
     f = synth.dbf_factors(3, 4096, 2048, 4096)
@@ -67,6 +67,24 @@ def test_dbf_general_r(ops, r, M):
     Y = _run(ops, xb, f, PATHS["auto"])
     ref = oracle.dbf_linear_chain(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"])
     assert_gemm_close(Y, ref, what=f"dbf r={r} M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_dbf_decode_with_the_smallest_workspace(ops, M):
+    # A workspace that holds only T (no room for the one-launch chain's barrier word) runs
+    # the two products as two launches; both give the oracle's result.
+    f = synth.dbf_factors(14 + M, 512, 256, 384)
+    xb, x = synth.activations(14, M, 384)
+    SB = ops.ob_pack_signs(_cuda(f["S_B"].astype(np.float32)))
+    SA = ops.ob_pack_signs(_cuda(f["S_A"].astype(np.float32)))
+    X = _cuda(xb.view(np.int16)).view(torch.bfloat16)
+    t_bytes = (M * 256 * 2 + 255) // 256 * 256
+    for ws_bytes in (t_bytes, ops.dbf_workspace_size(M, 256)):
+        ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+        Y = ops.dbf_linear(X, SB, _cuda(f["m"]), SA, _cuda(f["a"]), _cuda(f["b"]), workspace=ws)
+        torch.cuda.synchronize()
+        assert ops.ob_last_device_error() == 0
+        assert_gemm_close(Y, _ref(x, f), what=f"dbf M={M} workspace {ws_bytes}")
 
 
 def test_dbf_fp32_output(ops):

@@ -15,7 +15,7 @@ from helpers import assert_gemm_close, oracle_svid
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc_decode": 2, "tc": 3, "mma_decode": 4}
+PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "f8": 5}
 
 
 @pytest.fixture(scope="module")
@@ -171,8 +171,8 @@ def test_linear_degenerate_sizes(ops):
 
 # ---------------------------------------------------------------- full-size workloads
 
-@pytest.mark.parametrize("path", ["mma_decode", "tc_decode", "simt"])
-@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("path", ["mma_decode", "simt", "f8"])
+@pytest.mark.parametrize("M", [1, 2, 4, 16])
 def test_decode_workload_full(ops, path, M):
     # OneBit decode GEMV: X M x 4096, W 4096 x 4096 -> 2 MiB packed, a, b from SVID.
     W, a, b, _ = oracle_svid(1, 4096, 4096)
@@ -181,15 +181,24 @@ def test_decode_workload_full(ops, path, M):
     assert_gemm_close(Y, _ref(x, W, a, b), what=f"decode M={M} {path}")
 
 
-def test_prefill_workload_full_sampled_rows(ops):
-    # OneBit prefill: X 2048 x 4096, W 11008 x 4096; oracle on 64 sampled token rows.
+def test_prefill_workload_full_every_element(ops):
+    # OneBit prefill: X 2048 x 4096, W 11008 x 4096; all 22.5 M outputs against the fp64
+    # oracle (about 92 GFLOP on the host), on the path AUTO takes (the CTA-pair kernel).
+    W, a, b, _ = oracle_svid(2, 11008, 4096)
+    xb, x = synth.activations(2, 2048, 4096)
+    Y = _run(ops, xb, W, a, b, 0)
+    assert torch.isfinite(Y.float()).all()
+    assert_gemm_close(Y, _ref(x, W, a, b), what="prefill, every element")
+
+
+def test_prefill_one_cta_kernel_sampled_rows(ops):
+    # The one-CTA tcgen05 kernel on the prefill workload; oracle on 64 sampled token rows.
     W, a, b, _ = oracle_svid(2, 11008, 4096)
     xb, x = synth.activations(2, 2048, 4096)
     Y = _run(ops, xb, W, a, b, PATHS["tc"])
     rows = np.random.default_rng(0).choice(2048, 64, replace=False)
     rows[:2] = [0, 2047]
     assert_gemm_close(Y[torch.from_numpy(rows).cuda()], _ref(x[rows], W, a, b), what="prefill rows")
-    assert torch.isfinite(Y.float()).all()
 
 
 SWEEP = [(4096, 4096), (4096, 11008), (11008, 4096)]  # (K, N): K -> N
@@ -202,12 +211,8 @@ def test_sweep_with_outliers(ops, shape_idx, M):
     W, a, b, _ = oracle_svid(4 + shape_idx, N, K)
     xb, x = synth.activations(4 + shape_idx, M, K, outliers=True)
     Y = _run(ops, xb, W, a, b, 0)
-    if M <= 256:
-        assert_gemm_close(Y, _ref(x, W, a, b), what=f"sweep {K}->{N} M={M}")
-    else:
-        rows = np.random.default_rng(1).choice(M, 32, replace=False)
-        rows[:2] = [0, M - 1]
-        assert_gemm_close(Y[torch.from_numpy(rows).cuda()], _ref(x[rows], W, a, b), what=f"sweep rows M={M}")
+    # every element, M = 4096 included (up to 370 GFLOP of fp64 on the host)
+    assert_gemm_close(Y, _ref(x, W, a, b), what=f"sweep {K}->{N} M={M}")
 
 
 def test_cuda_graph_replay_matches(ops):
@@ -229,8 +234,9 @@ def test_cuda_graph_replay_matches(ops):
     assert_gemm_close(Y, _ref(x, W, a, b), what="graph replay")
 
 
-@pytest.mark.parametrize("M", [1, 4, 16, 40])
-def test_chained_layers_in_graph(ops, M):
+@pytest.mark.parametrize("M,path", [(1, "auto"), (4, "auto"), (16, "auto"), (40, "auto"), (1, "f8"), (3, "f8"),
+                                    (16, "f8")])
+def test_chained_layers_in_graph(ops, M, path):
     # Eight 512 x 512 layers chained through their outputs (layer i+1 reads layer i's Y),
     # captured in one CUDA graph; calls may launch before their predecessor has finished
     # (programmatic dependent launch), so each must read its input only after it is complete.
@@ -251,7 +257,7 @@ def test_chained_layers_in_graph(ops, M):
     def chain():
         x = X
         for (P, a, b), Y in zip(dev, Ys):
-            ops.ob_linear(x, P, a, b, out=Y, stream=s)
+            ops.ob_linear(x, P, a, b, out=Y, stream=s, path=PATHS.get(path, 0))
             x = Y
 
     with torch.cuda.stream(s):

@@ -14,7 +14,7 @@ from helpers import assert_gemm_close, oracle_svid
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"auto": 0, "simt": 1, "tc_decode": 2, "tc": 3, "mma_decode": 4}
+PATHS = {"auto": 0, "simt": 1, "tc": 3, "mma_decode": 4, "f8": 5}
 
 
 @pytest.fixture(scope="module")
@@ -44,7 +44,7 @@ def _svid32(W):
     return a.astype(np.float32), b.astype(np.float32)
 
 
-@pytest.mark.parametrize("path", ["simt", "tc_decode", "tc", "mma_decode"])
+@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "f8"])
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (4, 256, 256), (3, 200, 96), (17, 130, 160), (300, 264, 192)])
 def test_ln_small_shapes(ops, path, M, N, K):
     W = synth.weights(M + N + K, N, K)

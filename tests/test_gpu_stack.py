@@ -1,13 +1,10 @@
 """GPU parity of ob_linear_stack (a list of OneBit layers in one persistent launch).
 
 Every layer is checked against the fp64 oracle on the bf16 input it actually
-received (its X, possibly an earlier layer's Y), with the GEMM tolerances.  The
-warp-MMA kernel is the default; at one token OB_STACK_LUT=1 selects the table-lookup
-kernel where every layer's K is a multiple of 128 and the shares fit its staging
-buffer (the tests marked "lut" below set it).
+received (its X, possibly an earlier layer's Y), with the GEMM tolerances.  AUTO takes
+the fp8 form for one and two tokens and the bf16 warp-MMA form above; tests that name a
+path force one form.
 """
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -28,15 +25,7 @@ def ops():
     return _ops
 
 
-@pytest.fixture
-def lut_form():
-    old = os.environ.get("OB_STACK_LUT")
-    os.environ["OB_STACK_LUT"] = "1"
-    yield
-    if old is None:
-        del os.environ["OB_STACK_LUT"]
-    else:
-        os.environ["OB_STACK_LUT"] = old
+MMA, F8 = 4, 5
 
 
 def _cuda(x):
@@ -67,8 +56,8 @@ def _check(layers_host, layer_io, what):
         assert_gemm_close(Y, ref, what=f"{what} layer {i}")
 
 
-@pytest.mark.parametrize("M", [1, 4, 9, 16])
-def test_stack_chain(ops, M):
+@pytest.mark.parametrize("M,path", [(1, 0), (2, 0), (4, 0), (9, 0), (16, 0), (1, MMA), (2, MMA)])
+def test_stack_chain(ops, M, path):
     K = 512
     host = [_layer(200 + i, K, K) for i in range(8)]
     X0 = _x(synth.activations(200, M, K)[0])
@@ -77,27 +66,20 @@ def test_stack_chain(ops, M):
     for i, ((W, a, b), Y) in enumerate(zip(host, Ys)):
         spec.append((x, ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b), Y, i > 0))
         x = Y
-    ops.ob_linear_stack(spec, M)
+    ops.ob_linear_stack(spec, M, path=path)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
-    _check(host, [(s[0], s[4]) for s in spec], f"chain M={M}")
+    _check(host, [(s[0], s[4]) for s in spec], f"chain M={M} path={path}")
 
 
-def test_stack_chain_lut_form_one_token(ops, lut_form):
-    test_stack_chain(ops, 1)
-
-
-def test_stack_dbf_lut_form_one_token(ops, lut_form):
-    test_stack_dbf(ops, 1)
-
-
-def test_stack_lut_passes_and_segments(ops, lut_form):
-    # One token.  Group 1 (all read X0, K = 128): 60 layers of 32 rows (more layers than a
-    # CTA's segment slots, so the host checks every CTA's share; the first writes fp32),
-    # one of 30000 rows (about 203 rows per CTA: two passes of the table kernel), one of
-    # 1152 rows.  Group 2 reads the 1152-wide output: K = 1152 is one full 1024-k chunk
-    # and a 128-k tail; 300 rows, no input scale.
-    M = 1
+@pytest.mark.parametrize("M", [1, 2])
+def test_stack_f8_tiles_chunks_and_tails(ops, M):
+    # fp8 form.  Group 1 (all read X0, K = 128): 60 layers of 32 rows (a CTA's tile range
+    # crosses layers; the first writes fp32), one of 30000 rows (about 12.7 tiles per CTA:
+    # more than one 12-tile pass), one of 1152 rows.  Group 2 reads the 1152-wide output:
+    # K = 1152 is two full super-blocks and a 128-k tail; 300 rows (a ragged last tile), no
+    # input scale.  Group 3: a layer with K = 12832 (25 super-blocks and a tail: more than
+    # one staging chunk) on a separate input with outliers.
     X0 = _x(synth.activations(270, M, 128)[0])
     shapes = [(32, 128)] * 60 + [(30000, 128), (1152, 128), (300, 1152)]
     host, spec = [], []
@@ -108,13 +90,20 @@ def test_stack_lut_passes_and_segments(ops, lut_form):
         Y = torch.empty((M, N), dtype=torch.float32 if i == 0 else torch.bfloat16, device="cuda")
         X = spec[-1][4] if last else X0
         spec.append((X, ops.ob_pack_signs(_cuda(W)), _cuda(a), None if last else _cuda(b), Y, last))
-    ops.ob_linear_stack(spec, M)
+    # A long-K layer (25 super-blocks and a 32-k tail: two staging chunks), after a barrier.
+    Kl = 12832
+    W, a, b = _layer(399, 96, Kl)
+    host.append((W, a, b))
+    Xl = _x(synth.activations(271, M, Kl, outliers=True)[0])
+    spec.append((Xl, ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b),
+                 torch.empty((M, 96), dtype=torch.bfloat16, device="cuda"), True))
+    ops.ob_linear_stack(spec, M, path=F8)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
-    _check(host, [(sp[0], sp[4]) for sp in spec], "lut stack")
+    _check(host, [(sp[0], sp[4]) for sp in spec], f"f8 stack M={M}")
 
 
-@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("M", [1, 2, 5, 16])
 def test_stack_groups_ragged(ops, M):
     # Group 1 (independent, all read X0): A 96->224, B 96->130 (fp32 out), C 96->64 without input
     # scale.  Group 2 (after a barrier): D reads A (224->200), E reads A too (224->128, vector path).
@@ -138,8 +127,8 @@ def test_stack_groups_ragged(ops, M):
     _check([host[n] for n, _, _ in shapes], [(src[n], out[n]) for n, _, _ in shapes], f"groups M={M}")
 
 
-@pytest.mark.parametrize("M", [1, 16])
-def test_stack_dbf(ops, M):
+@pytest.mark.parametrize("M,path", [(1, 0), (2, 0), (16, 0), (1, MMA)])
+def test_stack_dbf(ops, M, path):
     # DBF as two layers: T = ((X ⊙ b) S_B^T) ⊙ m, then Y = (T S_A^T) ⊙ a (no input scale).
     f = synth.dbf_factors(220, 1024, 512, 768)
     xb, x = synth.activations(220, M, 768)
@@ -149,7 +138,7 @@ def test_stack_dbf(ops, M):
     SB = ops.ob_pack_signs(_cuda(f["S_B"].astype(np.float32)))
     SA = ops.ob_pack_signs(_cuda(f["S_A"].astype(np.float32)))
     ops.ob_linear_stack([(X, SB, _cuda(f["m"]), _cuda(f["b"]), T, False),
-                         (T, SA, _cuda(f["a"]), None, Y, True)], M)
+                         (T, SA, _cuda(f["a"]), None, Y, True)], M, path=path)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
     assert_gemm_close(Y, oracle.dbf_linear(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"]), what=f"dbf stack M={M}")
@@ -174,8 +163,9 @@ def test_stack_longer_than_one_launch(ops):
                           what=f"long stack layer {i}")
 
 
-def test_stack_in_cuda_graph(ops):
-    M, K = 4, 512
+@pytest.mark.parametrize("M", [1, 4])
+def test_stack_in_cuda_graph(ops, M):
+    K = 512
     host = [_layer(240 + i, K, K) for i in range(4)]
     X0 = _x(synth.activations(240, M, K)[0])
     Ys = [torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for _ in host]
@@ -201,20 +191,8 @@ def test_stack_in_cuda_graph(ops):
     _check(host, [(sp[0], sp[4]) for sp in spec], "graph stack")
 
 
-@pytest.mark.parametrize("M,lut", [(1, True), (1, False), (16, True)], ids=["M1", "M1-mma", "M16"])
-def test_stack_7b_block(ops, M, lut):
-    old = os.environ.get("OB_STACK_LUT")
-    os.environ["OB_STACK_LUT"] = "1" if lut else "0"
-    try:
-        _stack_7b_block(ops, M)
-    finally:
-        if old is None:
-            del os.environ["OB_STACK_LUT"]
-        else:
-            os.environ["OB_STACK_LUT"] = old
-
-
-def _stack_7b_block(ops, M):
+@pytest.mark.parametrize("M,path", [(1, 0), (1, MMA), (2, 0), (16, 0)], ids=["M1", "M1-mma", "M2", "M16"])
+def test_stack_7b_block(ops, M, path):
     # One 7B-shaped block: q, k, v, o (4096 -> 4096), gate, up (4096 -> 11008), down (11008 -> 4096).
     Wq, aq, bq, _ = oracle_svid(1, 4096, 4096)
     Wg, ag, bg, _ = oracle_svid(5, 11008, 4096)
@@ -230,7 +208,7 @@ def _stack_7b_block(ops, M):
     after = {"o": True, "gate": True, "down": True}
     order = ["q", "k", "v", "o", "gate", "up", "down"]
     spec = [(src[n], P[n][0], _cuda(P[n][1]), _cuda(P[n][2]), buf[n], after.get(n, False)) for n in order]
-    ops.ob_linear_stack(spec, M)
+    ops.ob_linear_stack(spec, M, path=path)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
     for n in order:
@@ -252,5 +230,9 @@ def test_stack_argument_errors(ops):
     with pytest.raises(ObError):  # workspace too small
         ops.ob_linear_stack([(X4, P, _cuda(a), _cuda(b), Y4, False)], 4,
                             workspace=torch.zeros(16, dtype=torch.uint8, device="cuda"))
+    with pytest.raises(ObError):  # the fp8 form takes at most two tokens
+        ops.ob_linear_stack([(X4, P, _cuda(a), _cuda(b), Y4, False)], 4, path=F8)
+    with pytest.raises(ObError):  # not a stack form
+        ops.ob_linear_stack([(X4, P, _cuda(a), _cuda(b), Y4, False)], 4, path=3)
     ops.ob_linear_stack([], 4)  # empty list: nothing to do
     assert ops.ob_last_device_error() == 0
