@@ -371,7 +371,7 @@ def run_ours(args, world, rank, local):
         return {"us_per_call": t * 1e6, "hbm_gbs": decode_call_bytes(m) / t / 1e9,
                 "frac_hbm": decode_call_bytes(m) / t / 1e9 / peaks["hbm_gbs"]}
 
-    for name, code in (("mma", ops.OB_PATH_MMA_DECODE), ("f8", ops.OB_PATH_F8), ("lut", ops.OB_PATH_SIMT)):
+    for name, code in (("mma", ops.OB_PATH_MMA_DECODE), ("i8", ops.OB_PATH_I8), ("lut", ops.OB_PATH_SIMT)):
         for m in DECODE_MS:
             if name == "lut" and m > 1:
                 continue
@@ -727,7 +727,7 @@ def run_stack(args, world, rank, local):
             pgraphs[m] = torch.cuda.CUDAGraph()
             with torch.cuda.graph(pgraphs[m], stream=stream):
                 ops.ob_linear_stack(specs[m], m, workspace=ws, stream=stream)
-        # The bf16 warp-MMA stack form forced at one token, beside the fp8 form AUTO takes.
+        # The bf16 warp-MMA stack form forced at one token, beside the int8 form AUTO takes.
         mgraphs = {}
         ops.ob_linear_stack(specs[1], 1, workspace=ws, stream=stream, path=ops.OB_PATH_MMA_DECODE)
         stream.synchronize()
@@ -773,7 +773,7 @@ def run_stack(args, world, rank, local):
                        "layers_per_token": calls, "weights_mb": wbytes / 1e6,
                        "l2": f"inputs larger than L2: {blocks * 7} distinct weight buffers ({wbytes / 1e6:.0f} MB)",
                        "graph": "one CUDA graph per token and M holding one ob_linear_stack (persistent, "
-                                "grid barriers between dependent layers; AUTO: fp8 form at M=1, bf16 warp-MMA "
+                                "grid barriers between dependent layers; AUTO: int8 form at M=1, bf16 warp-MMA "
                                 "form at M=16; persistent_bf16mma_M1 forces the bf16 form); per_call_* times one ob_linear "
                                 "per layer in a graph with programmatic dependent launch",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
@@ -784,6 +784,69 @@ def run_stack(args, world, rank, local):
     graphs.clear()
     pgraphs.clear()
     mgraphs.clear()
+
+
+SWEEP_SHAPES = ((4096, 4096), (4096, 11008), (11008, 4096))  # (K, N): the 7B-shaped outlier sweep
+SWEEP_MS = (1, 16, 256, 4096)
+
+
+def run_sweep(args, world, rank, local):
+    """The 7B-shaped layer sweep with outlier activations: K -> N in {4096 -> 4096,
+    4096 -> 11008, 11008 -> 4096} x M in {1, 16, 256, 4096}, through ob_linear (AUTO).
+
+    X ~ N(0, 1) bf16 with 6 fixed channels scaled x60 (the LLM.int8() page's outlier
+    features); W ~ N(0, 0.02) packed and SVID'd by the library.  M <= 16: one CUDA graph over
+    a pool of distinct weight copies larger than 3 x L2 (HBM-bound calls); M >= 256: rotating
+    input / output sets larger than L2.  Reports per (shape, M) the time per call, the HBM
+    fraction (packed weights + scales + X + Y bytes) and the dense bf16 fraction (2 M N K)."""
+    import torch
+    from binary_weight_gemm_b200 import build, synth
+    build.build()
+    from binary_weight_gemm_b200 import ops
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    peaks = load_peaks()
+    rows = {}
+    for si, (K, N) in enumerate(SWEEP_SHAPES):
+        W = torch.from_numpy(synth.weights(4 + si, N, K)).to(dev)
+        P = ops.ob_pack_signs(W, stream=stream)
+        a, b, _, _, _ = ops.ob_svid_rank1(W, stream=stream)
+        del W
+        wbytes = N * K // 8 + 4 * (N + K)
+        for M in SWEEP_MS:
+            X = torch.from_numpy(synth.activations(4 + si, M, K, outliers=True)[0].view(np.int16)).to(dev)
+            X = X.view(torch.bfloat16)
+            call_bytes = wbytes + 2 * M * K + 2 * M * N
+            if M <= 16:
+                nset = max(8, -(-3 * 126 * 2**20 // wbytes))
+                pool = [P.clone() for _ in range(nset)]
+                Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                t = _time_graph(lambda i: ops.ob_linear(X, pool[i % nset], a, b, out=Y, stream=stream), stream, nset)
+                del pool
+            else:
+                nset = max(2, -(-2 * 126 * 2**20 // (2 * M * (K + N))))
+                sets = [(X.clone(), torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for _ in range(nset)]
+                t = _time_calls(lambda i: ops.ob_linear(sets[i % nset][0], P, a, b, out=sets[i % nset][1],
+                                                        stream=stream), stream, max(10, 3 * nset))
+                del sets
+            fl = 2 * M * N * K
+            rows[f"{K}x{N}_M{M}"] = {"us_per_call": t * 1e6, "hbm_gbs": call_bytes / t / 1e9,
+                                     "frac_hbm": call_bytes / t / 1e9 / peaks["hbm_gbs"],
+                                     "tflops": fl / t / 1e12, "frac_bf16_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
+    if rank == 0:
+        tot_t = sum(r["us_per_call"] for r in rows.values()) * 1e-6
+        tot_fl = sum(2 * M * N * K for (K, N) in SWEEP_SHAPES for M in SWEEP_MS)
+        line = {
+            "metric": METRIC, "value": tot_fl / tot_t / 1e12, "unit": "TFLOP/s", "n_gpus": world, "steps": 1,
+            "warmup": 1, "ms_per_step": tot_t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "onebit_sweep_7b_outliers", "shapes_KxN": [list(x) for x in SWEEP_SHAPES],
+                       "M": list(SWEEP_MS), "outliers": "6 channels x60",
+                       "l2": "M<=16: weight pool > 3x L2 in one CUDA graph; M>=256: rotating sets > L2"},
+            "per_case": rows, "peak_source": peaks["source"], "gpu_launches": None, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
 
 
 def _time_calls(fn, stream, reps):
@@ -798,6 +861,29 @@ def _time_calls(fn, stream, reps):
         e1.record(stream)
         stream.synchronize()
     return e0.elapsed_time(e1) * 1e-3 / reps
+
+
+def _time_graph(fn, stream, reps, replays=5):
+    """Per-call time of fn(0 .. reps-1) captured in one CUDA graph (the deployed form: no host
+    launch overhead, programmatic dependent launch between kernels where the library uses it)."""
+    import torch
+    with torch.cuda.stream(stream):
+        fn(0)  # warm: kernel attributes, module load
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(reps):
+                fn(i)
+        g.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(replays):
+            g.replay()
+        e1.record(stream)
+        stream.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e-3 / (reps * replays)
 
 
 def run_extra(ops, dev, stream, peaks):
@@ -836,8 +922,8 @@ def run_extra(ops, dev, stream, peaks):
     for M in (1, 16):
         X = torch.from_numpy(synth.activations(1, M, 4096)[0].view(np.int16)).to(dev).view(torch.bfloat16)
         Y = torch.empty((M, 4096), dtype=torch.bfloat16, device=dev)
-        t0 = _time_calls(lambda i: ops.ob_linear(X, pool[i % 192], a1, b1, out=Y, stream=stream), stream, 384)
-        t1 = _time_calls(lambda i: ops.ob_linear_ln(X, pool[i % 192], a1, b1, out=Y, stream=stream), stream, 384)
+        t0 = _time_graph(lambda i: ops.ob_linear(X, pool[i % 192], a1, b1, out=Y, stream=stream), stream, 192)
+        t1 = _time_graph(lambda i: ops.ob_linear_ln(X, pool[i % 192], a1, b1, out=Y, stream=stream), stream, 192)
         out[f"decode_ln_M{M}"] = {"us_per_call": t1 * 1e6, "linear_only_us": t0 * 1e6, "ln_us": (t1 - t0) * 1e6,
                                   "hbm_gbs": decode_call_bytes(M) / t1 / 1e9}
     del pool
@@ -855,9 +941,10 @@ def run_extra(ops, dev, stream, peaks):
             X = torch.from_numpy(synth.activations(3, M, 4096)[0].view(np.int16)).to(dev).view(torch.bfloat16)
             Y = torch.empty((M, 4096), dtype=torch.bfloat16, device=dev)
             ws = torch.empty(ops.dbf_workspace_size(M, r), dtype=torch.uint8, device=dev)
-            t = _time_calls(lambda i: ops.dbf_linear(X, pool[i % nset][0], vec["m"], pool[i % nset][1], vec["a"],
-                                                     vec["b"], out=Y, workspace=ws, stream=stream), stream,
-                            max(50, 2 * nset))
+            timer = _time_graph if M <= 16 else _time_calls
+            t = timer(lambda i: ops.dbf_linear(X, pool[i % nset][0], vec["m"], pool[i % nset][1], vec["a"],
+                                               vec["b"], out=Y, workspace=ws, stream=stream), stream,
+                      max(50, 2 * nset))
             fl = 2 * M * r * (4096 + 4096)
             byts = wbytes + 4 * (4096 * 2 + r) + 2 * M * 4096 * 2
             key = f"dbf_M{M}" if r == 2048 else f"dbf_r{r}_M{M}"
@@ -875,10 +962,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "prefill", "stack", "factorize"], default="decode",
+    ap.add_argument("--workload", choices=["decode", "prefill", "stack", "factorize", "sweep"], default="decode",
                     help="decode: OneBit 4096x4096 at M=1,4,16 (default); prefill: M=2048, 4096 -> 11008; "
                          "stack: one token through 32 blocks of 7B-shaped OneBit layers at M=1 and 16; "
-                         "factorize: DBF factorisation of a 4096x4096 weight at r=2048")
+                         "factorize: DBF factorisation of a 4096x4096 weight at r=2048; "
+                         "sweep: the 7B-shaped layer sweep with outlier activations")
     ap.add_argument("--blocks", type=int, default=32, help="blocks of the stack workload")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-extra", dest="extra", action="store_false")
@@ -896,6 +984,8 @@ def main():
             run_stack(args, world, rank, local)
         elif args.workload == "factorize":
             run_factorize(args, world, rank, local)
+        elif args.workload == "sweep":
+            run_sweep(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -17,7 +17,7 @@ STATUS_NAMES = {
     9: "OB_ERR_UNSUPPORTED", 10: "OB_ERR_DEVICE_BOUNDS",
 }
 OB_OUT_BF16, OB_OUT_F32 = 0, 1
-OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC, OB_PATH_MMA_DECODE, OB_PATH_F8 = 0, 1, 3, 4, 5
+OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC, OB_PATH_MMA_DECODE, OB_PATH_I8 = 0, 1, 3, 4, 5
 
 
 

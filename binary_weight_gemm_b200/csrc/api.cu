@@ -93,7 +93,7 @@ ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) 
   switch (path) {
     case OB_PATH_SIMT: e = launch_sign_gemm_simt(g, c); break;
     case OB_PATH_MMA_DECODE: e = launch_sign_gemm_mma_decode(g, c); break;
-    case OB_PATH_F8: e = launch_sign_gemm_f8(g, c); break;
+    case OB_PATH_I8: e = launch_sign_gemm_i8(g, c); break;
     case OB_PATH_TC:
       // The CTA-pair kernel where it applies (bf16 Y, M >= 512, R >= 256, K <= 16384):
       // 1260 vs 1170 TFLOP/s for the one-CTA kernel at the prefill workload on B200.
@@ -106,9 +106,9 @@ ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Largest M the fp8 form of the layer stack takes (its activation limbs for up to two
+// Largest M the int8 form of the layer stack takes (its activation limbs for up to two
 // tokens fill one n8 tile).
-constexpr int64_t kStackF8MaxM = 2;
+constexpr int64_t kStackI8MaxM = 2;
 
 // Largest N, K or r of dbf_factorize: its GEMM grid has one row of CTAs per 128 rows, so
 // 2^22 rows keep grid.y at 32768, inside the 65535 limit.
@@ -202,7 +202,7 @@ ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
   if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
   if (!elems_ok(M, K) || !elems_ok(N, K) || !elems_ok(M, N)) return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
-  if (path < OB_PATH_AUTO || path > OB_PATH_F8 || path == 2) return OB_ERR_UNSUPPORTED;
+  if (path < OB_PATH_AUTO || path > OB_PATH_I8 || path == 2) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   if (K > 0 && (!X || !W_packed || !b)) return OB_ERR_NULL;
@@ -238,8 +238,8 @@ size_t ob_stack_workspace_size(void) { return 256; }
 ob_status ob_linear_stack_ex(const ob_layer* layers, int n_layers, int64_t M, void* workspace, size_t ws_bytes,
                              int path, void* stream) {
   if (n_layers < 0 || M < 0 || M > kDecodeMaxM) return OB_ERR_SHAPE;
-  if (path != OB_PATH_AUTO && path != OB_PATH_MMA_DECODE && path != OB_PATH_F8) return OB_ERR_UNSUPPORTED;
-  if (path == OB_PATH_F8 && M > kStackF8MaxM) return OB_ERR_UNSUPPORTED;
+  if (path != OB_PATH_AUTO && path != OB_PATH_MMA_DECODE && path != OB_PATH_I8) return OB_ERR_UNSUPPORTED;
+  if (path == OB_PATH_I8 && M > kStackI8MaxM) return OB_ERR_UNSUPPORTED;
   if (n_layers == 0 || M == 0) return OB_OK;
   if (!layers) return OB_ERR_NULL;
   if (!workspace) return OB_ERR_NULL;
@@ -260,7 +260,7 @@ ob_status ob_linear_stack_ex(const ob_layer* layers, int n_layers, int64_t M, vo
   LaunchCtx c;
   ob_status st = make_ctx(stream, &c);
   if (st != OB_OK) return st;
-  if (path == OB_PATH_AUTO) path = M <= kStackF8MaxM ? OB_PATH_F8 : OB_PATH_MMA_DECODE;
+  if (path == OB_PATH_AUTO) path = M <= kStackI8MaxM ? OB_PATH_I8 : OB_PATH_MMA_DECODE;
   return status_of(launch_sign_stack(host.data(), n_layers, M, static_cast<unsigned*>(workspace), c, path));
 }
 
@@ -300,7 +300,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   if (!elems_ok(M, K) || !elems_ok(r, K) || !elems_ok(M, r) || !elems_ok(N, r) || !elems_ok(M, N))
     return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
-  if (path < OB_PATH_AUTO || path > OB_PATH_F8 || path == 2) return OB_ERR_UNSUPPORTED;
+  if (path < OB_PATH_AUTO || path > OB_PATH_I8 || path == 2) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   const bool empty_sum = (K == 0 || r == 0);
@@ -328,7 +328,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
                                    {T, SA_packed, nullptr, a, Y, r, N, y_dtype, 1}};
     unsigned* bar = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + t_bytes);
     return status_of(
-        launch_sign_stack(two, 2, M, bar, c, M <= kStackF8MaxM ? OB_PATH_F8 : OB_PATH_MMA_DECODE));
+        launch_sign_stack(two, 2, M, bar, c, M <= kStackI8MaxM ? OB_PATH_I8 : OB_PATH_MMA_DECODE));
   }
   SignGemmArgs g1{static_cast<const uint16_t*>(X), M, K, SB_packed, r, b, m, T, r, OB_OUT_BF16};
   // Few output tiles (small M x r): split the first product over K into fp32 partial

@@ -5,7 +5,7 @@
 // reading the output of an earlier one.  Launched one kernel per layer, every
 // dependent layer pays a launch and a drain; here one cooperative grid walks the
 // whole list.  This file holds the bf16 warp-level MMA form (any M <= 16) and the
-// launcher, which takes the fp8 form of linear_stack_f8.cu for one or two tokens.
+// launcher, which takes the int8 form of linear_stack_i8.cu for one or two tokens.
 // The bf16 MMA form:
 //  * A layer flagged as reading an earlier layer's output waits at a grid-wide
 //    barrier; the layers between two barriers run back to back.
@@ -141,8 +141,8 @@ cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, un
     }
     e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned), c.stream);
     if (e != cudaSuccess) break;
-    if (path == OB_PATH_F8)
-      e = launch_stack_f8(*prm, c);
+    if (path == OB_PATH_I8 && stack_i8_supported(*prm))
+      e = launch_stack_i8(*prm, c);
     else
       e = M == 1 ? launch_stack_tok<1>(*prm, c) : (M <= 8 ? launch_stack_tok<8>(*prm, c) : launch_stack_tok<16>(*prm, c));
   }

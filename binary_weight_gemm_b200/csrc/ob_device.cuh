@@ -185,6 +185,15 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
                  : "memory");
 }
 
+// One untiled bulk copy global -> this CTA's shared memory (no multicast), completing
+// `bytes` transaction bytes on `bar`.  Both addresses 16-byte aligned, bytes a multiple
+// of 16.
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // One warp prefetches a contiguous block into L2 in 4 KB pieces, one piece per lane
 // at a time.  base must be 16-byte aligned.
 __device__ __forceinline__ void prefetch_block_l2(const void* base, uint64_t bytes, int lane) {

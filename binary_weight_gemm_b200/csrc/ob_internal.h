@@ -37,8 +37,8 @@ cudaError_t launch_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* ou
 
 cudaError_t launch_sign_gemm_simt(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_mma_decode(const SignGemmArgs& g, const LaunchCtx& c);
-// fp8 tensor-core sign product for small M (linear_f8.cu, f8_block.cuh).
-cudaError_t launch_sign_gemm_f8(const SignGemmArgs& g, const LaunchCtx& c);
+// int8 tensor-core sign product for one or two tokens per pass (linear_i8.cu, i8_block.cuh).
+cudaError_t launch_sign_gemm_i8(const SignGemmArgs& g, const LaunchCtx& c);
 cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c);
 // cuTensorMapEncodeTiled from the driver (null if unavailable).
 void* tensor_map_encode_tiled_fn();
@@ -87,8 +87,8 @@ struct StackLayerHost {
   int barrier;          // reads an output of an earlier layer of the list
 };
 // Runs the list (M <= 16) as cooperative launches of at most stack_max_layers_per_launch()
-// layers; bar: 8 bytes of device memory (zeroed by the launcher).  path: OB_PATH_F8 (M <= 2)
-// for the fp8 form, OB_PATH_MMA_DECODE for the bf16 form.
+// layers; bar: 8 bytes of device memory (zeroed by the launcher).  path: OB_PATH_I8 (M <= 2)
+// for the int8 form, OB_PATH_MMA_DECODE for the bf16 form.
 cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c,
                               int path);
 int stack_max_layers_per_launch();

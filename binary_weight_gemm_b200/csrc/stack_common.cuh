@@ -1,6 +1,6 @@
 // stack_common.cuh -- the layer list and the grid-wide barrier of the persistent
 // layer-stack kernels (linear_stack.cu: bf16 warp-level MMA blocks, any M <= 16;
-// linear_stack_f8.cu: fp8 warp-level MMA on staged activation limbs, M <= 2).
+// linear_stack_i8.cu: int8 warp-level MMA on staged activation limbs, M <= 2).
 //
 // Each layer is  Y = [(X ⊙ b^T) W_sign^T] ⊙ a^T  ("1bit量化", blog.zerodtree.com,
 // "proposition 1").  A layer flagged `barrier` reads an output of an earlier layer
@@ -38,8 +38,10 @@ struct StackParams {
   StackLayer L[kStackMaxLayers];
 };
 
-// The one- and two-token fp8 tensor-core stack (linear_stack_f8.cu).
-cudaError_t launch_stack_f8(const StackParams& p, const LaunchCtx& c);
+// The one- and two-token int8 tensor-core stack (linear_stack_i8.cu): M <= 2 and one
+// 16-row tile of every layer fits its 80 KB weight buffer (K <= 40960).
+bool stack_i8_supported(const StackParams& p);
+cudaError_t launch_stack_i8(const StackParams& p, const LaunchCtx& c);
 
 #ifdef __CUDACC__
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {

@@ -15,7 +15,7 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import (OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_F8, OB_PATH_MMA_DECODE, OB_PATH_SIMT,  # noqa: F401
+from ._lib import (OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_I8, OB_PATH_MMA_DECODE, OB_PATH_SIMT,  # noqa: F401
                    OB_PATH_TC, ObError)
 
 
@@ -139,7 +139,7 @@ def ob_linear_stack(layers, M: int, workspace: torch.Tensor | None = None, strea
     layers: sequence of (X, W_packed, a, b, Y, after_previous); X bf16 [M, K], W_packed int32
     [N, K/32], a fp32 [N], b fp32 [K] or None, Y bf16/fp32 [M, N] (written), after_previous:
     True if X is an output of an earlier layer of the list.  path: OB_PATH_AUTO,
-    OB_PATH_MMA_DECODE or OB_PATH_F8 (M <= 2).
+    OB_PATH_MMA_DECODE or OB_PATH_I8 (M <= 2).
     """
     arr = (_lib.ObLayer * max(1, len(layers)))()
     dev = None

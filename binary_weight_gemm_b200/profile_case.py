@@ -4,7 +4,7 @@
     python -m binary_weight_gemm_b200.profile_case prefill --reps 6
     python -m binary_weight_gemm_b200.profile_case dbf --m 512 --reps 6
     python -m binary_weight_gemm_b200.profile_case stack --m 1 --blocks 8 --reps 5
-    python -m binary_weight_gemm_b200.profile_case stack --m 1 --chain 128 --reps 5 --path f8
+    python -m binary_weight_gemm_b200.profile_case stack --m 1 --chain 128 --reps 5 --path i8
 
 The workloads are the benchmark's: OneBit 4096 x 4096 decode at M tokens, OneBit
 prefill X 2048 x 4096 -> 11008, DBF K = N = 4096 with r = 2048, and the layer stack:
@@ -46,12 +46,12 @@ def main(argv=None) -> None:
     ap.add_argument("--reps", type=int, default=6)
     ap.add_argument("--blocks", type=int, default=8, help="stack: 7B-shaped blocks")
     ap.add_argument("--chain", type=int, default=0, help="stack: chained 1024 -> 1024 layers instead")
-    ap.add_argument("--path", choices=("auto", "mma", "f8"), default="auto",
-                    help="stack / decode: kernel form (AUTO, the bf16 warp MMA, or the fp8 form)")
+    ap.add_argument("--path", choices=("auto", "mma", "i8"), default="auto",
+                    help="stack / decode: kernel form (AUTO, the bf16 warp MMA, or the int8 form)")
     args = ap.parse_args(argv)
     dev = torch.device("cuda", 0)
     torch.cuda.init()
-    path = {"auto": ops.OB_PATH_AUTO, "mma": ops.OB_PATH_MMA_DECODE, "f8": ops.OB_PATH_F8}[args.path]
+    path = {"auto": ops.OB_PATH_AUTO, "mma": ops.OB_PATH_MMA_DECODE, "i8": ops.OB_PATH_I8}[args.path]
 
     if args.case in ("decode", "prefill"):
         M, N, K = (args.m or 16, 4096, 4096) if args.case == "decode" else (args.m or 2048, 11008, 4096)

@@ -89,8 +89,9 @@ typedef enum ob_path {
   OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA); K <= 32768; a
                               2-CTA (cta_group::2) tile where bf16 Y, M >= 512, N >= 256, K <= 16384 */
   OB_PATH_MMA_DECODE = 4,  /* bf16 warp-level MMA, signs unpacked in registers, M <= 16 per pass */
-  OB_PATH_F8 = 5           /* fp8 (e4m3) warp-level MMA: each packed word becomes eight operand registers
-                              with one AND each, activations in three e4m3 limbs; M <= 16 per pass */
+  OB_PATH_I8 = 5           /* int8 warp-level MMA (u8 x s8 -> s32): each packed word becomes eight operand
+                              registers with one AND each, activations quantised per token to 21 bits in
+                              three 7-bit limbs, exact integer sums; M <= 2 per pass */
 } ob_path;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -225,15 +226,16 @@ OB_API size_t ob_stack_workspace_size(void);
  *              concurrently running ob_linear_stack.
  * Weights and scales must not be outputs of layers of the same list.  Validation of
  * every descriptor happens before anything is launched.  Asynchronous.
- * Kernel (OB_PATH_AUTO): M <= 2, the fp8 form (one contiguous range of 16-row tiles
- * per CTA and barrier group, activation limbs staged once per layer per CTA, e4m3
- * warp-level MMA); M > 2, the bf16 warp-level MMA form (32-row blocks round robin).
+ * Kernel (OB_PATH_AUTO): M <= 2, the int8 form (one contiguous range of 16-row tiles
+ * per CTA and barrier group, packed signs fetched into shared memory by bulk copies ahead
+ * of the grid barrier, activation limbs staged once per layer per CTA, u8 x s8 warp-level
+ * MMA); M > 2, the bf16 warp-level MMA form (32-row blocks round robin).
  */
 OB_API ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M,
                           void* workspace, size_t ws_bytes, void* stream);
 
 /* ob_linear_stack with an explicit form: OB_PATH_AUTO, OB_PATH_MMA_DECODE (bf16, any
- * M <= 16) or OB_PATH_F8 (M <= 2; OB_ERR_UNSUPPORTED above).  Other values:
+ * M <= 16) or OB_PATH_I8 (M <= 2; OB_ERR_UNSUPPORTED above).  Other values:
  * OB_ERR_UNSUPPORTED. */
 OB_API ob_status ob_linear_stack_ex(const ob_layer* layers, int n_layers, int64_t M,
                              void* workspace, size_t ws_bytes, int path, void* stream);
@@ -264,7 +266,7 @@ OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
  *              products (it stays in L2 at the workload sizes).
  * K % 32 == 0, r % 32 == 0.  Asynchronous.  M <= 16 (decode): both products run in
  * one persistent launch (the layer-stack kernels with a grid barrier between the two
- * products; fp8 form for M <= 2), so T never leaves the chip's L2 between them; larger
+ * products; int8 form for M <= 2), so T never leaves the chip's L2 between them; larger
  * M: two tcgen05 GEMMs.
  */
 OB_API ob_status dbf_linear(const void* X, int64_t M, int64_t K,

@@ -53,3 +53,27 @@ def header_functions(path: str) -> list[str]:
             if m:
                 names.append(m.group(1))
     return names
+
+
+CANARY_BYTE = 0xA5
+CANARY_PAD = 4096  # bytes before and after; keeps the interior 256-byte aligned
+
+
+class Guarded:
+    """A CUDA tensor inside a larger allocation whose CANARY_PAD bytes on each side hold
+    CANARY_BYTE, so that a kernel writing past either end of its output is caught
+    (compute-sanitizer is not available; this is the stand-in for output buffers)."""
+
+    def __init__(self, shape, dtype, device="cuda"):
+        import torch
+        nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self._buf = torch.full((CANARY_PAD + nbytes + CANARY_PAD,), CANARY_BYTE, dtype=torch.uint8, device=device)
+        self._n = nbytes
+        self.t = self._buf[CANARY_PAD:CANARY_PAD + nbytes].view(dtype).view(shape)
+
+    def check(self, what=""):
+        head = self._buf[:CANARY_PAD]
+        tail = self._buf[CANARY_PAD + self._n:]
+        bad_h = int((head != CANARY_BYTE).sum())
+        bad_t = int((tail != CANARY_BYTE).sum())
+        assert bad_h == 0 and bad_t == 0, f"{what}: {bad_h} bytes before and {bad_t} bytes after the buffer overwritten"

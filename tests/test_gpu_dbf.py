@@ -5,11 +5,11 @@ import torch
 
 import oracle
 from binary_weight_gemm_b200 import synth
-from helpers import assert_gemm_close
+from helpers import Guarded, assert_gemm_close
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "f8": 5, "auto": 0}
+PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5, "auto": 0}
 
 
 @pytest.fixture(scope="module")
@@ -29,9 +29,15 @@ def _run(ops, xb, f, path, out_dtype=torch.bfloat16):
     SB = ops.ob_pack_signs(_cuda(f["S_B"].astype(np.float32)))
     SA = ops.ob_pack_signs(_cuda(f["S_A"].astype(np.float32)))
     X = _cuda(xb.view(np.int16)).view(torch.bfloat16)
-    Y = ops.dbf_linear(X, SB, _cuda(f["m"]), SA, _cuda(f["a"]), _cuda(f["b"]), out_dtype=out_dtype, path=path)
+    M, r, N = xb.shape[0], SB.shape[0], SA.shape[0]
+    g = Guarded((M, N), out_dtype)
+    ws = Guarded((max(1, ops.dbf_workspace_size(M, r)),), torch.uint8)
+    Y = ops.dbf_linear(X, SB, _cuda(f["m"]), SA, _cuda(f["a"]), _cuda(f["b"]), out_dtype=out_dtype, path=path,
+                       out=g.t, workspace=ws.t)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
+    g.check("dbf_linear output")
+    ws.check("dbf_linear workspace")
     return Y
 
 
@@ -39,7 +45,7 @@ def _ref(x, f):
     return oracle.dbf_linear(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"])
 
 
-@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "f8", "auto"])
+@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "i8", "auto"])
 @pytest.mark.parametrize("M,N,r,K", [(1, 128, 32, 64), (4, 256, 96, 256), (7, 200, 160, 96), (33, 130, 64, 128),
                                      (260, 256, 128, 320)])
 def test_dbf_small_shapes(ops, path, M, N, r, K):

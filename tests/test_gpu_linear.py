@@ -11,11 +11,11 @@ import torch
 
 import oracle
 from binary_weight_gemm_b200 import synth
-from helpers import assert_gemm_close, oracle_svid
+from helpers import Guarded, assert_gemm_close, oracle_svid
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "f8": 5}
+PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5}
 
 
 @pytest.fixture(scope="module")
@@ -37,9 +37,11 @@ def _x_bf16(x_bits):
 
 def _run(ops, x_bits, W, a, b, path, out_dtype=torch.bfloat16):
     P = ops.ob_pack_signs(_cuda(W))
-    Y = ops.ob_linear(_x_bf16(x_bits), P, _cuda(a), _cuda(b), out_dtype=out_dtype, path=path)
+    g = Guarded((x_bits.shape[0], W.shape[0]), out_dtype)
+    Y = ops.ob_linear(_x_bf16(x_bits), P, _cuda(a), _cuda(b), out_dtype=out_dtype, path=path, out=g.t)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
+    g.check("ob_linear output")
     return Y
 
 
@@ -171,7 +173,7 @@ def test_linear_degenerate_sizes(ops):
 
 # ---------------------------------------------------------------- full-size workloads
 
-@pytest.mark.parametrize("path", ["mma_decode", "simt", "f8"])
+@pytest.mark.parametrize("path", ["mma_decode", "simt", "i8"])
 @pytest.mark.parametrize("M", [1, 2, 4, 16])
 def test_decode_workload_full(ops, path, M):
     # OneBit decode GEMV: X M x 4096, W 4096 x 4096 -> 2 MiB packed, a, b from SVID.
@@ -234,8 +236,8 @@ def test_cuda_graph_replay_matches(ops):
     assert_gemm_close(Y, _ref(x, W, a, b), what="graph replay")
 
 
-@pytest.mark.parametrize("M,path", [(1, "auto"), (4, "auto"), (16, "auto"), (40, "auto"), (1, "f8"), (3, "f8"),
-                                    (16, "f8")])
+@pytest.mark.parametrize("M,path", [(1, "auto"), (4, "auto"), (16, "auto"), (40, "auto"), (1, "i8"), (2, "i8"), (3, "i8"),
+                                    (16, "i8")])
 def test_chained_layers_in_graph(ops, M, path):
     # Eight 512 x 512 layers chained through their outputs (layer i+1 reads layer i's Y),
     # captured in one CUDA graph; calls may launch before their predecessor has finished

@@ -10,11 +10,11 @@ import torch
 
 import oracle
 from binary_weight_gemm_b200 import synth
-from helpers import assert_gemm_close, oracle_svid
+from helpers import Guarded, assert_gemm_close, oracle_svid
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"auto": 0, "simt": 1, "tc": 3, "mma_decode": 4, "f8": 5}
+PATHS = {"auto": 0, "simt": 1, "tc": 3, "mma_decode": 4, "i8": 5}
 
 
 @pytest.fixture(scope="module")
@@ -33,9 +33,11 @@ def _cuda(x):
 def _run(ops, xb, W, a, b, path=0, eps=1e-5, out_dtype=torch.bfloat16):
     P = ops.ob_pack_signs(_cuda(W))
     X = _cuda(xb.view(np.int16)).view(torch.bfloat16)
-    Z = ops.ob_linear_ln(X, P, _cuda(a), _cuda(b), eps=eps, out_dtype=out_dtype, path=path)
+    g = Guarded((xb.shape[0], W.shape[0]), out_dtype)
+    Z = ops.ob_linear_ln(X, P, _cuda(a), _cuda(b), eps=eps, out_dtype=out_dtype, path=path, out=g.t)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
+    g.check("ob_linear_ln output")
     return Z
 
 
@@ -44,7 +46,7 @@ def _svid32(W):
     return a.astype(np.float32), b.astype(np.float32)
 
 
-@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "f8"])
+@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "i8"])
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (4, 256, 256), (3, 200, 96), (17, 130, 160), (300, 264, 192)])
 def test_ln_small_shapes(ops, path, M, N, K):
     W = synth.weights(M + N + K, N, K)

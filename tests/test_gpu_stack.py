@@ -2,7 +2,7 @@
 
 Every layer is checked against the fp64 oracle on the bf16 input it actually
 received (its X, possibly an earlier layer's Y), with the GEMM tolerances.  AUTO takes
-the fp8 form for one and two tokens and the bf16 warp-MMA form above; tests that name a
+the int8 form for one and two tokens and the bf16 warp-MMA form above; tests that name a
 path force one form.
 """
 import numpy as np
@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from binary_weight_gemm_b200 import synth
-from helpers import assert_gemm_close, oracle_svid
+from helpers import Guarded, assert_gemm_close, oracle_svid
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +25,7 @@ def ops():
     return _ops
 
 
-MMA, F8 = 4, 5
+MMA, I8 = 4, 5
 
 
 def _cuda(x):
@@ -61,20 +61,22 @@ def test_stack_chain(ops, M, path):
     K = 512
     host = [_layer(200 + i, K, K) for i in range(8)]
     X0 = _x(synth.activations(200, M, K)[0])
-    Ys = [torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for _ in host]
+    gs = [Guarded((M, K), torch.bfloat16) for _ in host]
     spec, x = [], X0
-    for i, ((W, a, b), Y) in enumerate(zip(host, Ys)):
-        spec.append((x, ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b), Y, i > 0))
-        x = Y
+    for i, ((W, a, b), g) in enumerate(zip(host, gs)):
+        spec.append((x, ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b), g.t, i > 0))
+        x = g.t
     ops.ob_linear_stack(spec, M, path=path)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
+    for i, g in enumerate(gs):
+        g.check(f"chain layer {i} output")
     _check(host, [(s[0], s[4]) for s in spec], f"chain M={M} path={path}")
 
 
 @pytest.mark.parametrize("M", [1, 2])
-def test_stack_f8_tiles_chunks_and_tails(ops, M):
-    # fp8 form.  Group 1 (all read X0, K = 128): 60 layers of 32 rows (a CTA's tile range
+def test_stack_i8_tiles_chunks_and_tails(ops, M):
+    # int8 form.  Group 1 (all read X0, K = 128): 60 layers of 32 rows (a CTA's tile range
     # crosses layers; the first writes fp32), one of 30000 rows (about 12.7 tiles per CTA:
     # more than one 12-tile pass), one of 1152 rows.  Group 2 reads the 1152-wide output:
     # K = 1152 is two full super-blocks and a 128-k tail; 300 rows (a ragged last tile), no
@@ -97,10 +99,10 @@ def test_stack_f8_tiles_chunks_and_tails(ops, M):
     Xl = _x(synth.activations(271, M, Kl, outliers=True)[0])
     spec.append((Xl, ops.ob_pack_signs(_cuda(W)), _cuda(a), _cuda(b),
                  torch.empty((M, 96), dtype=torch.bfloat16, device="cuda"), True))
-    ops.ob_linear_stack(spec, M, path=F8)
+    ops.ob_linear_stack(spec, M, path=I8)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
-    _check(host, [(sp[0], sp[4]) for sp in spec], f"f8 stack M={M}")
+    _check(host, [(sp[0], sp[4]) for sp in spec], f"i8 stack M={M}")
 
 
 @pytest.mark.parametrize("M", [1, 2, 5, 16])
@@ -230,8 +232,8 @@ def test_stack_argument_errors(ops):
     with pytest.raises(ObError):  # workspace too small
         ops.ob_linear_stack([(X4, P, _cuda(a), _cuda(b), Y4, False)], 4,
                             workspace=torch.zeros(16, dtype=torch.uint8, device="cuda"))
-    with pytest.raises(ObError):  # the fp8 form takes at most two tokens
-        ops.ob_linear_stack([(X4, P, _cuda(a), _cuda(b), Y4, False)], 4, path=F8)
+    with pytest.raises(ObError):  # the int8 form takes at most two tokens
+        ops.ob_linear_stack([(X4, P, _cuda(a), _cuda(b), Y4, False)], 4, path=I8)
     with pytest.raises(ObError):  # not a stack form
         ops.ob_linear_stack([(X4, P, _cuda(a), _cuda(b), Y4, False)], 4, path=3)
     ops.ob_linear_stack([], 4)  # empty list: nothing to do
