@@ -16,6 +16,14 @@
 // GEMV writes per-split partial sums that a second kernel adds in a fixed
 // order, so the iteration itself is deterministic; only the fp64 norm
 // accumulators use atomics.
+//
+// The stopping test runs on the device: the last block of each iteration's
+// update kernel decides whether the iteration converged (or met a NaN) and
+// sets a flag that turns every later kernel of the loop into a no-op.  The host
+// queues iterations in batches of kBatch followed by the final pass, and reads
+// the outcome back once per batch: once in all, when the iteration converges
+// within the first batch.
+#include <algorithm>
 #include <cmath>
 
 #include "ob_device.cuh"
@@ -27,12 +35,23 @@ namespace {
 constexpr int kSplitsMax = 64;
 constexpr int kColThreads = 256;
 
+constexpr int kBatch = 8;  // iterations queued between two reads of the outcome
+
 struct SvidScalars {
-  double yy;     // ||y||^2 of the current iteration
-  double diff2;  // ||v_new - v||^2
-  double zz;     // ||z||^2 in the final pass
-  double pad;
+  double yy;         // ||y||^2 of the current iteration
+  double diff2;      // ||v_new - v||^2 of the current iteration
+  double zz;         // ||z||^2 in the final pass
+  unsigned arrived;  // blocks of the current update kernel that have added their share
+  int state;         // kRunning, kConverged or kNan
+  int iters;         // iterations completed
+  int pad;
 };
+
+constexpr int kRunning = 0, kConverged = 1, kNan = 2;
+
+__device__ __forceinline__ int svid_state(const SvidScalars* sc) {
+  return *reinterpret_cast<const volatile int*>(&sc->state);
+}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -56,9 +75,18 @@ __global__ void svid_init_kernel(float* v, int64_t K) {
 
 // z[n] = sum_k |W[n,k]| v[k]; one warp per row, float4 loads.  If zz != null,
 // also accumulates ||z||^2.
+// final == false: an iteration's pass, skipped once the loop has stopped.  final == true:
+// the pass after the loop (zz = ||z||^2), run when it converged, or at the cap (force).
+__device__ __forceinline__ bool svid_skip(const SvidScalars* sc, bool final, bool force) {
+  const int st = svid_state(sc);
+  return final ? !(st == kConverged || (force && st == kRunning)) : st != kRunning;
+}
+
 __global__ void __launch_bounds__(256) svid_rowdot_kernel(const float* __restrict__ W, int64_t N, int64_t K,
                                                           const float* __restrict__ v, float* __restrict__ z,
-                                                          double* zz) {
+                                                          SvidScalars* sc, bool final, bool force) {
+  if (svid_skip(sc, final, force)) return;
+  double* zz = final ? &sc->zz : nullptr;
   const int lane = threadIdx.x & 31;
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -85,7 +113,8 @@ __global__ void __launch_bounds__(256) svid_rowdot_kernel(const float* __restric
 __global__ void __launch_bounds__(kColThreads) svid_coldot_kernel(const float* __restrict__ W, int64_t N,
                                                                    int64_t K, const float* __restrict__ z,
                                                                    float* __restrict__ part,
-                                                                   int64_t rows_per_split) {
+                                                                   int64_t rows_per_split, const SvidScalars* sc) {
+  if (svid_skip(sc, false, false)) return;
   const int64_t k = blockIdx.x * (int64_t)kColThreads + threadIdx.x;
   const int64_t s = blockIdx.y;
   const int64_t n0 = s * rows_per_split;
@@ -123,6 +152,7 @@ __device__ __forceinline__ double block_sum(double x, double* red) {
 // y[k] = sum_s part[s][k] in a fixed order; accumulates ||y||^2.
 __global__ void __launch_bounds__(256) svid_colsum_kernel(const float* __restrict__ part, int splits, int64_t K,
                                                           float* __restrict__ y, SvidScalars* sc) {
+  if (svid_skip(sc, false, false)) return;
   __shared__ double red[8];
   double local = 0.0;
   for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < K; k += (int64_t)gridDim.x * blockDim.x) {
@@ -135,11 +165,14 @@ __global__ void __launch_bounds__(256) svid_colsum_kernel(const float* __restric
   if (threadIdx.x == 0) atomicAdd(&sc->yy, t);
 }
 
-// v <- y / ||y||; accumulates ||v_new - v||^2.  ||y|| == 0 leaves v unchanged.
+// v <- y / ||y||; accumulates ||v_new - v||^2.  ||y|| == 0 leaves v unchanged.  The last
+// block to finish takes the stopping decision and clears the accumulators for the next
+// iteration (every block has read yy before it arrives).
 __global__ void __launch_bounds__(256) svid_update_kernel(const float* __restrict__ y, float* __restrict__ v,
-                                                          int64_t K, SvidScalars* sc) {
+                                                          int64_t K, SvidScalars* sc, double tol2) {
+  if (svid_skip(sc, false, false)) return;
   __shared__ double red[8];
-  const double yy = sc->yy;
+  const double yy = *reinterpret_cast<const volatile double*>(&sc->yy);
   double local = 0.0;
   if (yy > 0.0) {
     const float inv = (float)(1.0 / sqrt(yy));
@@ -152,12 +185,28 @@ __global__ void __launch_bounds__(256) svid_update_kernel(const float* __restric
     }
   }
   const double t = block_sum(local, red);
-  if (threadIdx.x == 0) atomicAdd(&sc->diff2, t);
+  if (threadIdx.x == 0) {
+    atomicAdd(&sc->diff2, t);
+    __threadfence();
+    if (atomicAdd(&sc->arrived, 1u) == gridDim.x - 1) {
+      __threadfence();
+      const double d2 = *reinterpret_cast<const volatile double*>(&sc->diff2);
+      sc->iters += 1;
+      if (isnan(yy) || isnan(d2))
+        sc->state = kNan;
+      else if (!(yy > 0.0) || d2 <= tol2)  // an all-zero |W| stops at once
+        sc->state = kConverged;
+      sc->yy = 0.0;
+      sc->diff2 = 0.0;
+      sc->arrived = 0u;
+    }
+  }
 }
 
 // a = z / sqrt(sigma1), b = sqrt(sigma1) v, sigma1 = ||z||.
 __global__ void svid_finish_kernel(const float* __restrict__ z, const float* __restrict__ v, int64_t N, int64_t K,
-                                   const SvidScalars* sc, float* a, float* b, float* sigma1) {
+                                   const SvidScalars* sc, float* a, float* b, float* sigma1, bool force) {
+  if (svid_skip(sc, true, force)) return;
   const double s = sqrt(sc->zz);
   const bool zero = !(s > 0.0);
   const float ra = zero ? 0.f : (float)(1.0 / sqrt(s));
@@ -192,43 +241,36 @@ ob_status run_svid(const float* W, int64_t N, int64_t K, float* a, float* b, flo
   const int64_t rows_per_split = (N + splits - 1) / splits;
   splits = (N + rows_per_split - 1) / rows_per_split;
 
+  if (cudaMemsetAsync(sc, 0, sizeof(SvidScalars), st) != cudaSuccess) return OB_ERR_CUDA;
   svid_init_kernel<<<vec_blocks, 256, 0, st>>>(v, K);
   if (cudaGetLastError() != cudaSuccess) return OB_ERR_CUDA;
 
   const double tol2 = (double)tol * (double)tol;
-  bool converged = false;
-  int it = 0;
-  while (it < max_iters) {
-    ++it;
-    if (cudaMemsetAsync(sc, 0, sizeof(SvidScalars), st) != cudaSuccess) return OB_ERR_CUDA;
-    svid_rowdot_kernel<<<row_blocks, 256, 0, st>>>(W, N, K, v, z, nullptr);
-    svid_coldot_kernel<<<dim3((unsigned)stripes, (unsigned)splits), kColThreads, 0, st>>>(W, N, K, z, part,
-                                                                                        rows_per_split);
-    svid_colsum_kernel<<<vec_blocks, 256, 0, st>>>(part, (int)splits, K, y, sc);
-    svid_update_kernel<<<vec_blocks, 256, 0, st>>>(y, v, K, sc);
+  int queued = 0;
+  for (;;) {
+    const int nb = std::min(kBatch, max_iters - queued);
+    for (int i = 0; i < nb; ++i) {
+      svid_rowdot_kernel<<<row_blocks, 256, 0, st>>>(W, N, K, v, z, sc, false, false);
+      svid_coldot_kernel<<<dim3((unsigned)stripes, (unsigned)splits), kColThreads, 0, st>>>(W, N, K, z, part,
+                                                                                          rows_per_split, sc);
+      svid_colsum_kernel<<<vec_blocks, 256, 0, st>>>(part, (int)splits, K, y, sc);
+      svid_update_kernel<<<vec_blocks, 256, 0, st>>>(y, v, K, sc, tol2);
+    }
+    queued += nb;
+    const bool force = queued >= max_iters;  // the cap: finish with the last iterate
+    svid_rowdot_kernel<<<row_blocks, 256, 0, st>>>(W, N, K, v, z, sc, true, force);
+    svid_finish_kernel<<<vec_blocks, 256, 0, st>>>(z, v, N, K, sc, a, b, sigma1, force);
     if (cudaGetLastError() != cudaSuccess) return OB_ERR_CUDA;
     SvidScalars host;
     if (cudaMemcpyAsync(&host, sc, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess) return OB_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return OB_ERR_CUDA;
-    if (std::isnan(host.yy) || std::isnan(host.diff2)) {
-      if (iters_out) *iters_out = it;
-      return OB_ERR_NAN;
-    }
-    if (!(host.yy > 0.0) || host.diff2 <= tol2) {  // all-zero |W| converges at once
-      converged = true;
-      break;
+    if (iters_out) *iters_out = host.iters;
+    if (host.state == kNan) return OB_ERR_NAN;
+    if (host.state == kConverged || force) {
+      if (std::isnan(host.zz)) return OB_ERR_NAN;
+      return host.state == kConverged ? OB_OK : OB_ERR_NOT_CONVERGED;
     }
   }
-  if (cudaMemsetAsync(sc, 0, sizeof(SvidScalars), st) != cudaSuccess) return OB_ERR_CUDA;
-  svid_rowdot_kernel<<<row_blocks, 256, 0, st>>>(W, N, K, v, z, &sc->zz);
-  svid_finish_kernel<<<vec_blocks, 256, 0, st>>>(z, v, N, K, sc, a, b, sigma1);
-  if (cudaGetLastError() != cudaSuccess) return OB_ERR_CUDA;
-  SvidScalars host;
-  if (cudaMemcpyAsync(&host, sc, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess) return OB_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return OB_ERR_CUDA;
-  if (iters_out) *iters_out = it;
-  if (std::isnan(host.zz)) return OB_ERR_NAN;
-  return converged ? OB_OK : OB_ERR_NOT_CONVERGED;
 }
 
 }  // namespace ob

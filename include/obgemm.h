@@ -135,7 +135,9 @@ OB_API size_t ob_svid_workspace_size(int64_t N, int64_t K);
  *   tol        stop when ||v_t - v_{t-1}||_2 <= tol (<= 0 selects 1e-6).
  *   iters_out  HOST int, or NULL: iterations taken.
  *   workspace  device, at least ob_svid_workspace_size(N, K) bytes.
- * Synchronises `stream` once per iteration (it is an offline conversion).
+ * The stopping test runs on the device; the host queues 8 iterations at a time and
+ * synchronises `stream` once per 8 (once in all when the iteration converges within
+ * 8, as it does on the workloads in 3); it is an offline conversion.
  * Returns OB_ERR_NOT_CONVERGED with the last iterate written if the cap is
  * reached, OB_ERR_NAN if W holds NaN.  An all-zero W gives a = b = 0,
  * sigma1 = 0 and OB_OK.
