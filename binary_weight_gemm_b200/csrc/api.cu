@@ -202,7 +202,10 @@ ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
   if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
   if (!elems_ok(M, K) || !elems_ok(N, K) || !elems_ok(M, N)) return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
-  if (path < OB_PATH_AUTO || path > OB_PATH_I8 || path == 2) return OB_ERR_UNSUPPORTED;
+  if (path < 0 || (path & ~0xFF & ~OB_FLAG_STATIC_WEIGHTS) != 0) return OB_ERR_UNSUPPORTED;
+  const int static_w = (path & OB_FLAG_STATIC_WEIGHTS) ? 1 : 0;
+  path &= 0xFF;
+  if (path > OB_PATH_I8 || path == 2) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   if (K > 0 && (!X || !W_packed || !b)) return OB_ERR_NULL;
@@ -213,6 +216,7 @@ ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
   if (st != OB_OK) return st;
   if (K == 0) return zero_output(Y, M, N, y_dtype, c.stream);
   SignGemmArgs g{static_cast<const uint16_t*>(X), M, K, W_packed, N, b, a, Y, N, y_dtype};
+  g.static_w = static_w;
   return run_sign_gemm(g, path, c);
 }
 
@@ -300,7 +304,10 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   if (!elems_ok(M, K) || !elems_ok(r, K) || !elems_ok(M, r) || !elems_ok(N, r) || !elems_ok(M, N))
     return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
-  if (path < OB_PATH_AUTO || path > OB_PATH_I8 || path == 2) return OB_ERR_UNSUPPORTED;
+  if (path < 0 || (path & ~0xFF & ~OB_FLAG_STATIC_WEIGHTS) != 0) return OB_ERR_UNSUPPORTED;
+  const int static_w = (path & OB_FLAG_STATIC_WEIGHTS) ? 1 : 0;
+  path &= 0xFF;
+  if (path > OB_PATH_I8 || path == 2) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   const bool empty_sum = (K == 0 || r == 0);

@@ -18,11 +18,12 @@
 //    q = l0 + 128 l1 + 16384 l2 (l0, l1 in [0, 128), l2 in [-64, 64]).  Column n = 3 m + l of
 //    the B operand holds limb l of token m.  The rounding is the only approximation (2^-21
 //    of the chunk's largest |x'|).
-//  * A (16 rows x 32 k, weights): register R_j = w & (0x01010101 << j) of a packed word w
-//    holds, in byte i, bit 8i + j of w left at bit j: the u8 value 2^j bit.  One MMA takes
-//    a single position j from two packed words (a0/a1 from word 2p, a2/a3 from word 2p+1
-//    of the lane's four), so all its A values are multiples of 2^j; it accumulates into
-//    chain j, and sum_j (acc_j >> j) is the exact integer sum of bit * limb.
+//  * A (16 rows x 32 k, weights): for bit position j = 2i + c (i = 0..3, c = 0, 1) the
+//    register (w >> 2i) & (0x01010101 << c) of a packed word w holds, in byte i', bit
+//    8i' + j of w at bit c: the u8 value 2^c bit (one shift per word and i, one AND per
+//    four weights).  One MMA takes a single position j from two packed words (a0/a1 from
+//    word 2p, a2/a3 from word 2p+1 of the lane's four) and accumulates into chain (p, c):
+//    four chains, whose sum of acc >> c is the exact integer sum of bit * limb.
 //  * The integer sums are converted and scaled, -2 * 128^l / sigma per column, when a
 //    tile's share of a chunk is done; T is added in the epilogue.
 //
@@ -201,18 +202,33 @@ __device__ __forceinline__ void stage_quantise(const StageRaw& raw, int m, int s
   }
 }
 
+// Chains per tile: (p, c) with p the word pair and c the parity of the bit position.
+constexpr int kChains = 4;
+
+// The A registers of bit position j = 2i + c from the shifted words (word >> 2i).
+__device__ __forceinline__ void mma_pos(int (&acc)[4], uint32_t g0, uint32_t h0, uint32_t g1, uint32_t h1, int c,
+                                        uint2 b) {
+  const uint32_t msk = 0x01010101u << c;
+  mma_u8s8(acc, g0 & msk, h0 & msk, g1 & msk, h1 & msk, b.x, b.y);
+}
+
 // One tile's rows g / g+8 (packed words wg / wh: words 4t .. 4t+3 of the super-block)
-// times staged super-block s, accumulated into the eight position chains.
-__device__ __forceinline__ void tile_sb(const uint32_t* fr, uint4 wg, uint4 wh, int (&acc)[8][4], int lane) {
+// times staged super-block s, accumulated into the four chains.
+__device__ __forceinline__ void tile_sb(const uint32_t* fr, uint4 wg, uint4 wh, int (&acc)[kChains][4], int lane) {
   const uint32_t g4[4] = {wg.x, wg.y, wg.z, wg.w};
   const uint32_t h4[4] = {wh.x, wh.y, wh.z, wh.w};
 #pragma unroll
   for (int p = 0; p < 2; ++p)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t msk = 0x01010101u << j;
-      const uint2 b = *reinterpret_cast<const uint2*>(fr + ((p * 8 + j) * 32 + lane) * 2);
-      mma_u8s8(acc[j], g4[2 * p] & msk, h4[2 * p] & msk, g4[2 * p + 1] & msk, h4[2 * p + 1] & msk, b.x, b.y);
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t g0 = g4[2 * p] >> (2 * i), h0 = h4[2 * p] >> (2 * i);
+      const uint32_t g1 = g4[2 * p + 1] >> (2 * i), h1 = h4[2 * p + 1] >> (2 * i);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int j = 2 * i + c;
+        const uint2 b = *reinterpret_cast<const uint2*>(fr + ((p * 8 + j) * 32 + lane) * 2);
+        mma_pos(acc[2 * p + c], g0, h0, g1, h1, c, b);
+      }
     }
 }
 
@@ -230,25 +246,24 @@ __device__ __forceinline__ void load_sb_regs(const uint32_t* fr, int lane, SbReg
 }
 
 // tile_sb with the super-block's fragments already in registers.
-__device__ __forceinline__ void tile_sb_regs(const SbRegs& fr, uint4 wg, uint4 wh, int (&acc)[8][4]) {
+__device__ __forceinline__ void tile_sb_regs(const SbRegs& fr, uint4 wg, uint4 wh, int (&acc)[kChains][4]) {
   const uint32_t g4[4] = {wg.x, wg.y, wg.z, wg.w};
   const uint32_t h4[4] = {wh.x, wh.y, wh.z, wh.w};
 #pragma unroll
   for (int p = 0; p < 2; ++p)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t msk = 0x01010101u << j;
-      mma_u8s8(acc[j], g4[2 * p] & msk, h4[2 * p] & msk, g4[2 * p + 1] & msk, h4[2 * p + 1] & msk, fr.b[p][j].x,
-               fr.b[p][j].y);
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t g0 = g4[2 * p] >> (2 * i), h0 = h4[2 * p] >> (2 * i);
+      const uint32_t g1 = g4[2 * p + 1] >> (2 * i), h1 = h4[2 * p + 1] >> (2 * i);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) mma_pos(acc[2 * p + c], g0, h0, g1, h1, c, fr.b[p][2 * i + c]);
     }
 }
 
-// sum_j (acc_j >> j) for accumulator register r: the exact integer sum of bit * limb.
-__device__ __forceinline__ int combine(const int (&acc)[8][4], int r) {
-  int s = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) s += acc[j][r] >> j;
-  return s;
+// sum over the chains of acc >> c for accumulator register r: the exact integer sum of
+// bit * limb.
+__device__ __forceinline__ int combine(const int (&acc)[kChains][4], int r) {
+  return (acc[0][r] + acc[2][r]) + ((acc[1][r] + acc[3][r]) >> 1);
 }
 
 // The fold factors of the chunk's columns: -2 * 128^l / sigma_m for column 3 m + l (0 for

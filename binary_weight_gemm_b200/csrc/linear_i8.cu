@@ -114,9 +114,9 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_i8_kernel(SignGemmArgs g, 
     }
     __syncthreads();
     // Multiply: exact int32 sums per bit position over the warp's items, folded once.
-    int acc[8][4];
+    int acc[kChains][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < kChains; ++j)
 #pragma unroll
       for (int r = 0; r < 4; ++r) acc[j][r] = 0;
 #pragma unroll

@@ -56,16 +56,19 @@ __global__ void __launch_bounds__(kThreads, TOK > 8 ? 1 : 2) sign_gemm_mma_decod
   __shared__ BlockShared<TOK> shb;
   const int64_t n0 = (int64_t)blockIdx.x * kRowsPerCta;
   // Before the previous grid has finished, only pull this CTA's sign rows (one
-  // contiguous block) into L2; the reads themselves come after pdl_wait.
+  // contiguous block) into L2; the reads themselves come after pdl_wait.  With static
+  // weights (the previous grid did not write them) each warp's first chunk of sign
+  // words is requested into shared memory already.
   if (g.l2_prefetch && threadIdx.x < 32 && n0 < g.R) {
     const int64_t Wd = g.K / 32;
     const int64_t rows = min64(kRowsPerCta, g.R - n0);
     prefetch_block_l2(g.S + n0 * Wd, (uint64_t)(rows * Wd) * 4u, threadIdx.x);
     if (g.iscale) prefetch_block_l2(g.iscale, (uint64_t)g.K * 4u, threadIdx.x);
   }
+  if (g.static_w) fetch_words(g, n0, kVec, warp_words<TOK>(dsm, threadIdx.x >> 5), threadIdx.x >> 5, 0, threadIdx.x & 31);
   pdl_wait();  // every input may have been written by the previous grid in the stream
   pdl_launch_dependents();  // the next grid may start (one grid ahead at most)
-  block<TOK, false>(g, m0, n0, kVec, dsm, shb);
+  block<TOK, false>(g, m0, n0, kVec, dsm, shb, g.static_w != 0);
 }
 
 template <int TOK, bool kVec>

@@ -162,12 +162,27 @@ __global__ void __launch_bounds__(kSimtThreads) sign_gemv_simt_kernel(SignGemmAr
   }
 }
 
-// Single-token kernel: one CTA per 32-row table-lookup block (lut_block.cuh).
-template <int Q>
+// Single-token kernel: one CTA per 32-row table-lookup block (lut_block.cuh).  With
+// static weights (kStatic: the previous grid did not write S or the scales) the first
+// chunk's sign words and the output scales are loaded before the programmatic-launch
+// wait, so that they stream in while the previous grid finishes.
+template <int Q, bool kStatic>
 __global__ void __launch_bounds__(kSimtThreads) sign_gemv_lut_kernel(SignGemmArgs g, int64_t m0) {
   extern __shared__ float lut[];
+  const int64_t row_base = (int64_t)blockIdx.x * lutb::kRowsPerBlock;
+  const int64_t row0 = lutb::warp_row0(row_base);
+  uint32_t wq[lutb::kRowsPerWarp][Q];
+  float osc[lutb::kRowsPerWarp];
+  if constexpr (kStatic) {
+    lutb::load_signs<Q>(g, row0, 0, wq, threadIdx.x & 31);
+    lutb::load_oscale(g, row0, osc);
+  }
   prologue_wait();
-  lutb::block<Q, false>(g, m0, (int64_t)blockIdx.x * lutb::kRowsPerBlock, lut);
+  if constexpr (!kStatic) {
+    lutb::load_signs<Q>(g, row0, 0, wq, threadIdx.x & 31);
+    lutb::load_oscale(g, row0, osc);
+  }
+  lutb::block<Q, false>(g, m0, row_base, lut, wq, osc);
 }
 
 // Launch with programmatic stream serialization when enabled: the kernel may
@@ -193,7 +208,7 @@ cudaError_t launch_pdl(Kern kern, int64_t blocks, size_t smem, const SignGemmArg
 template <int Q>
 cudaError_t launch_lut(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c) {
   const size_t smem = sizeof(float) * 16 * 32 * Q * 8;
-  auto kern = sign_gemv_lut_kernel<Q>;
+  auto kern = g.static_w ? sign_gemv_lut_kernel<Q, true> : sign_gemv_lut_kernel<Q, false>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -137,6 +137,16 @@ __device__ __forceinline__ Seg first_seg(const Sched& sc, int gi) {
   return Seg{-1, 0, 0};
 }
 
+// One thread: request the scale vectors of segment s (of layer L) into L2: the input scale
+// is read by the staging right after a grid barrier, the output scale by the epilogue.
+__device__ void prefetch_scales(const StackLayer& L, const Seg& s) {
+  const int64_t r0 = s.t0 * 16, r1 = min64((s.t0 + s.nt) * 16, L.N);
+  if (L.iscale)
+    for (int64_t off = 0; off < L.K * 4; off += 4096) prefetch_l2_bulk(reinterpret_cast<const char*>(L.iscale) + off,
+                                                                      (uint32_t)min64(4096, L.K * 4 - off));
+  prefetch_l2_bulk(L.oscale + r0, (uint32_t)((r1 - r0) * 4));
+}
+
 // One thread: request the packed rows of segment s (of layer L) into the buffer.  The bulk
 // copy takes the largest multiple of 16 bytes; the at most three words after it are copied
 // by this thread first, so that the arrival (a release) publishes them with the phase.
@@ -152,12 +162,7 @@ __device__ void fetch_seg(const StackLayer& L, const Seg& s, uint32_t* wbuf, uin
   fence_proxy_async_smem();
   mbar_arrive_expect_tx(bar, bulk);
   if (bulk) bulk_g2s(wbuf, src, bulk, bar);
-  // The segment's scale vectors into L2 as well: the input scale is read by the staging
-  // right after the next grid barrier, the output scale by the epilogue.
-  if (L.iscale)
-    for (int64_t off = 0; off < L.K * 4; off += 4096) prefetch_l2_bulk(reinterpret_cast<const char*>(L.iscale) + off,
-                                                                      (uint32_t)min64(4096, L.K * 4 - off));
-  prefetch_l2_bulk(L.oscale + r0, (uint32_t)((r1 - r0) * 4));
+  prefetch_scales(L, s);
 }
 
 // The last warp copies layer li's descriptor from the parameter block into shared memory
@@ -361,9 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
               ng = smem_words(wbuf, Wd, 16 * (i + 1) + gq, nrows, w0, L.vec != 0);
               nh = smem_words(wbuf, Wd, 16 * (i + 1) + gq + 8, nrows, w0, L.vec != 0);
             }
-            int acc[8][4];
+            int acc[kChains][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < kChains; ++j)
 #pragma unroll
               for (int r = 0; r < 4; ++r) acc[j][r] = 0;
             if (s < chn) tile_sb_regs(fr, wg, wh, acc);
@@ -380,9 +385,9 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
         } else if (!s_abort) {
           const float f0 = st.fcol[2 * tq], f1 = st.fcol[2 * tq + 1];
           for (int i = 0; i < sg.nt; ++i) {
-            int acc[8][4];
+            int acc[kChains][4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < kChains; ++j)
 #pragma unroll
               for (int r = 0; r < 4; ++r) acc[j][r] = 0;
             for (int s = warp; s < chn; s += kWarps) {

@@ -8,8 +8,7 @@
 // costs one shared-memory load and one add instead of four select/adds.  Table
 // layout: entry v of group (lane group c, word q, nibble j) sits at
 // v * 32*Q*8 + (8q + j) * 32 + c, so lane c always reads bank c.  8 warps x 4 rows.
-// Used by the per-call one-token kernel (one CTA per block) and by the layer-stack
-// kernel (persistent CTAs walking a list of blocks).
+// Used by the per-call one-token kernel (one CTA per block).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -41,36 +40,60 @@ __device__ __forceinline__ uint2 load_x8(const uint16_t* p) {
     return __ldg(reinterpret_cast<const uint2*>(p));
 }
 
+// This lane's sign words of chunk c0 (32 lanes x Q words) for the warp's rows starting at row0.
+template <int Q>
+__device__ __forceinline__ void load_signs(const SignGemmArgs& g, int64_t row0, int64_t c0,
+                                           uint32_t (&wq)[kRowsPerWarp][Q], int lane) {
+  const int64_t Wd = g.K / 32, G = (Wd + Q - 1) / Q;
+  const int64_t grp = c0 + lane;
+#pragma unroll
+  for (int r = 0; r < kRowsPerWarp; ++r) {
+    const int64_t n = row0 + r;
+    const bool ok = n < g.R && grp < G;
+    const uint32_t* srow = g.S + (ok ? n : 0) * Wd;
+    if constexpr (Q == 4) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (ok) v = __ldcs(reinterpret_cast<const uint4*>(srow) + grp);
+      wq[r][0] = v.x; wq[r][1] = v.y; wq[r][2] = v.z; wq[r][3] = v.w;
+    } else {
+      wq[r][0] = ok ? __ldcs(srow + grp) : 0u;
+    }
+  }
+}
+
+// The output scales of the warp's rows.
+__device__ __forceinline__ void load_oscale(const SignGemmArgs& g, int64_t row0, float (&osc)[kRowsPerWarp]) {
+#pragma unroll
+  for (int r = 0; r < kRowsPerWarp; ++r) osc[r] = (row0 + r < g.R) ? __ldg(g.oscale + row0 + r) : 0.f;
+}
+
+// First row of the calling warp's rows in a block.
+__device__ __forceinline__ int64_t warp_row0(int64_t row_base) { return row_base + (threadIdx.x >> 5) * kRowsPerWarp; }
+
 // Y[m0, row_base .. row_base + 31]; all 256 threads call it; it ends with __syncthreads().
+// wq0: the lane's sign words of the first chunk and osc: the output scales, both loaded by
+// the caller with load_signs / load_oscale (before or after the programmatic-launch wait).
 template <int Q, bool kCoherentX>
-__device__ __forceinline__ void block(const SignGemmArgs& g, int64_t m0, int64_t row_base, float* lut) {
+__device__ __forceinline__ void block(const SignGemmArgs& g, int64_t m0, int64_t row_base, float* lut,
+                                      const uint32_t (&wq0)[kRowsPerWarp][Q], const float (&osc)[kRowsPerWarp]) {
   constexpr int kGroups = 32 * Q * 8;  // nibble groups per chunk (4 k each)
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const int64_t K = g.K, Wd = K / 32, G = (Wd + Q - 1) / Q;
-  const int64_t row0 = row_base + warp * kRowsPerWarp;
+  const int64_t row0 = warp_row0(row_base);
   float acc[kRowsPerWarp];
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) acc[r] = 0.f;
-  float osc[kRowsPerWarp];
-#pragma unroll
-  for (int r = 0; r < kRowsPerWarp; ++r) osc[r] = (row0 + r < g.R) ? __ldg(g.oscale + row0 + r) : 0.f;
 
   for (int64_t c0 = 0; c0 < G; c0 += 32) {
     // 1. This lane's sign words for every row of the warp.
     uint32_t wq[kRowsPerWarp][Q];
-    const int64_t grp = c0 + lane;
+    if (c0 == 0) {
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-      const int64_t n = row0 + r;
-      const bool ok = n < g.R && grp < G;
-      const uint32_t* srow = g.S + (ok ? n : 0) * Wd;
-      if constexpr (Q == 4) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (ok) v = __ldcs(reinterpret_cast<const uint4*>(srow) + grp);
-        wq[r][0] = v.x; wq[r][1] = v.y; wq[r][2] = v.z; wq[r][3] = v.w;
-      } else {
-        wq[r][0] = ok ? __ldcs(srow + grp) : 0u;
-      }
+      for (int r = 0; r < kRowsPerWarp; ++r)
+#pragma unroll
+        for (int q = 0; q < Q; ++q) wq[r][q] = wq0[r][q];
+    } else {
+      load_signs<Q>(g, row0, c0, wq, lane);
     }
     // 2. Tabulate this chunk: thread t builds groups with c = t % 32, (8q+j) = t/32 + 8i.
     constexpr int kPerThread = kGroups / kThreads;  // 4 (Q = 4) or 1 (Q = 1)

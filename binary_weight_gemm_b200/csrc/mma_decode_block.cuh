@@ -81,15 +81,57 @@ struct BlockShared {
   alignas(16) uint32_t bt[kWarps][kChunkWords][2][8];  // input-scale pairs per (word, step, t)
 };
 
+// The calling warp's word tiles (two buffers of 32 rows x 16 words) in the block's
+// dynamic shared memory.
+template <int TOK>
+__device__ __forceinline__ uint32_t* warp_words(uint8_t* dsm, int warp) {
+  constexpr int NN = TOK > 8 ? 2 : 1;
+  uint32_t* swbase = reinterpret_cast<uint32_t*>(dsm + sizeof(uint2) * kWarps * kChunkWords * 2 * NN * 32);
+  return swbase + warp * 2 * kRowsPerCta * kChunkWords;
+}
+
+// Request the calling warp's sign words of a chunk (32 rows x 16 words) into buffer `buf`
+// of its word tiles `sw` (one cp.async group).
+__device__ __forceinline__ void fetch_words(const SignGemmArgs& g, int64_t n0, bool vec, uint32_t* sw, int64_t chunk,
+                                            int buf, int lane) {
+  const int64_t Wd = g.K / 32;
+  const int64_t nchunks = (Wd + kChunkWords - 1) / kChunkWords;
+  uint32_t* dst = sw + buf * kRowsPerCta * kChunkWords;
+  const int64_t w0 = chunk * kChunkWords;
+  if (vec) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // 32 rows x 4 groups of 4 words = 128 copies per warp
+      const int item = lane + 32 * i;
+      const int row = item >> 2, q = item & 3;
+      const int64_t n = n0 + row;
+      const bool ok = n < g.R && chunk < nchunks && w0 + 4 * q < Wd;
+      const uint32_t* src = g.S + (ok ? n * Wd + w0 + 4 * q : 0);
+      cp_async16(dst + word_slot(row, 4 * q), src, ok);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {  // 32 rows x 16 single words
+      const int item = lane + 32 * i;
+      const int row = item >> 4, w = item & 15;
+      const int64_t n = n0 + row;
+      const bool ok = n < g.R && chunk < nchunks && w0 + w < Wd;
+      const uint32_t* src = g.S + (ok ? n * Wd + w0 + w : 0);
+      cp_async4(dst + word_slot(row, w), src, ok);
+    }
+  }
+  cp_async_commit();
+}
+
 // Y rows n0 .. n0+31 for tokens m0 .. m0+min(TOK, M-m0)-1.  All 256 threads call
 // it; it ends with __syncthreads().  vec: the sign rows allow 16-byte copies.
+// first_fetched: the caller has already issued fetch_words for each warp's first chunk
+// (chunk = warp, buffer 0), e.g. before a programmatic-launch wait.
 template <int TOK, bool kCoherentX>
 __device__ __forceinline__ void block(const SignGemmArgs& g, int64_t m0, int64_t n0, bool vec, uint8_t* dsm,
-                                      BlockShared<TOK>& shb) {
+                                      BlockShared<TOK>& shb, bool first_fetched = false) {
   constexpr int NN = TOK > 8 ? 2 : 1;
   constexpr int TOKN = TOK > 8 ? 8 : TOK;  // real tokens staged per n8 tile
   auto fb = reinterpret_cast<uint2 (*)[kChunkWords][2][NN][32]>(dsm);
-  uint32_t* swbase = reinterpret_cast<uint32_t*>(dsm + sizeof(uint2) * kWarps * kChunkWords * 2 * NN * 32);
   auto& red = shb.red;
   auto& bt = shb.bt;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -97,35 +139,8 @@ __device__ __forceinline__ void block(const SignGemmArgs& g, int64_t m0, int64_t
   const int64_t K = g.K, Wd = K / 32;
   const int64_t mt = min64(TOK, g.M - m0);
   const int64_t nchunks = (Wd + kChunkWords - 1) / kChunkWords;
-  uint32_t* sw = swbase + warp * 2 * kRowsPerCta * kChunkWords;
-
-  // Request this warp's sign words of a chunk (32 rows x 16 words) into buffer `buf`.
-  auto fetch_words = [&](int64_t chunk, int buf) {
-    uint32_t* dst = sw + buf * kRowsPerCta * kChunkWords;
-    const int64_t w0 = chunk * kChunkWords;
-    if (vec) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {  // 32 rows x 4 groups of 4 words = 128 copies per warp
-        const int item = lane + 32 * i;
-        const int row = item >> 2, q = item & 3;
-        const int64_t n = n0 + row;
-        const bool ok = n < g.R && chunk < nchunks && w0 + 4 * q < Wd;
-        const uint32_t* src = g.S + (ok ? n * Wd + w0 + 4 * q : 0);
-        cp_async16(dst + word_slot(row, 4 * q), src, ok);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {  // 32 rows x 16 single words
-        const int item = lane + 32 * i;
-        const int row = item >> 4, w = item & 15;
-        const int64_t n = n0 + row;
-        const bool ok = n < g.R && chunk < nchunks && w0 + w < Wd;
-        const uint32_t* src = g.S + (ok ? n * Wd + w0 + w : 0);
-        cp_async4(dst + word_slot(row, w), src, ok);
-      }
-    }
-    cp_async_commit();
-  };
+  uint32_t* sw = warp_words<TOK>(dsm, warp);
+  auto fetch = [&](int64_t chunk, int buf) { fetch_words(g, n0, vec, sw, chunk, buf, lane); };
 
   // Stage one chunk for this warp: the B fragments (the activations, copied into
   // fragment order, no arithmetic) and the input-scale pairs that the A
@@ -201,14 +216,14 @@ __device__ __forceinline__ void block(const SignGemmArgs& g, int64_t m0, int64_t
         for (int i = 0; i < 4; ++i) acc[q][rt][nn][i] = 0.f;
 
   int64_t chunk = warp;
-  fetch_words(chunk, 0);
+  if (!first_fetched) fetch(chunk, 0);
   const int my_row = tid & (kRowsPerCta - 1);  // the output row this thread stores
   const float osc = (n0 + my_row < g.R) ? __ldg(g.oscale + n0 + my_row) : 0.f;
   int buf = 0;
   for (; chunk < nchunks; chunk += kWarps, buf ^= 1) {
     stage_x(chunk);
     if (chunk + kWarps < nchunks) {
-      fetch_words(chunk + kWarps, buf ^ 1);
+      fetch(chunk + kWarps, buf ^ 1);
       asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's words have landed
     } else {
       cp_async_wait_all();

@@ -31,6 +31,8 @@ struct SignGemmArgs {
   int64_t ldy;
   int y_dtype;          // ob_out_dtype
   int l2_prefetch;      // set by the dispatcher: prefetch this launch's weights into L2 first
+  int static_w;         // S, iscale and oscale were not written by the previous grid in the
+                        // stream: kernels may read them before the programmatic-launch wait
 };
 
 cudaError_t launch_pack_signs(const float* W, int64_t N, int64_t K, uint32_t* out, const LaunchCtx& c);

@@ -1,6 +1,6 @@
 """Run one kernel case a fixed number of times, for profiling under ncu.
 
-    python -m binary_weight_gemm_b200.profile_case decode --m 16 --reps 40
+    python -m binary_weight_gemm_b200.profile_case decode --m 16 --reps 40 [--static]
     python -m binary_weight_gemm_b200.profile_case prefill --reps 6
     python -m binary_weight_gemm_b200.profile_case dbf --m 512 --reps 6
     python -m binary_weight_gemm_b200.profile_case stack --m 1 --blocks 8 --reps 5
@@ -48,10 +48,13 @@ def main(argv=None) -> None:
     ap.add_argument("--chain", type=int, default=0, help="stack: chained 1024 -> 1024 layers instead")
     ap.add_argument("--path", choices=("auto", "mma", "i8"), default="auto",
                     help="stack / decode: kernel form (AUTO, the bf16 warp MMA, or the int8 form)")
+    ap.add_argument("--static", action="store_true",
+                    help="decode: OR OB_FLAG_STATIC_WEIGHTS into the path (as the benchmark's decode calls do)")
     args = ap.parse_args(argv)
     dev = torch.device("cuda", 0)
     torch.cuda.init()
     path = {"auto": ops.OB_PATH_AUTO, "mma": ops.OB_PATH_MMA_DECODE, "i8": ops.OB_PATH_I8}[args.path]
+    lin_path = path | (ops.OB_FLAG_STATIC_WEIGHTS if args.static else 0)
 
     if args.case in ("decode", "prefill"):
         M, N, K = (args.m or 16, 4096, 4096) if args.case == "decode" else (args.m or 2048, 11008, 4096)
@@ -68,7 +71,7 @@ def main(argv=None) -> None:
 
         def call(i):
             X, P, a, b, Y = sets[i % n_sets]
-            ops.ob_linear(X, P, a, b, out=Y, path=path)
+            ops.ob_linear(X, P, a, b, out=Y, path=lin_path)
     elif args.case == "stack":
         M = args.m or 1
         if args.chain:
@@ -128,7 +131,8 @@ def main(argv=None) -> None:
     assert ops.ob_last_device_error() == 0
     if args.case != "stack":
         desc = {"N": N, "K": K}
-    print(json.dumps({"case": args.case, "M": M, **desc, "path": args.path, "reps": args.reps, "sets": n_sets,
+    print(json.dumps({"case": args.case, "M": M, **desc, "path": args.path, "static": args.static, "reps": args.reps,
+                      "sets": n_sets,
                       "us_per_call": e0.elapsed_time(e1) * 1e3 / args.reps}))
 
 

@@ -94,6 +94,16 @@ typedef enum ob_path {
                               three 7-bit limbs, exact integer sums; M <= 2 per pass */
 } ob_path;
 
+/* Flag OR-ed into the path argument of ob_linear_ex (and ob_linear_ln): the caller
+ * guarantees that W_packed, a and b were not written by the kernel launched just before
+ * this call on the same stream (weights loaded once and used by call after call).  The
+ * one-token kernel (its sign words and output scales) and the warp-MMA decode kernel (its
+ * first chunk of sign words) then start reading before waiting for that kernel to finish
+ * (programmatic dependent launch), so the weights stream in while it runs.  The other
+ * kernels ignore the flag.  Any other bit above the low 8 is rejected with
+ * OB_ERR_UNSUPPORTED. */
+#define OB_FLAG_STATIC_WEIGHTS 0x100
+
 /* Human-readable name of a status code (static string, never NULL). */
 OB_API const char* ob_status_string(int status);
 

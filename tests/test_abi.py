@@ -75,6 +75,10 @@ def test_host_argument_checks_without_gpu(lib):
     # options
     assert lib.ob_linear(p, 1, 64, p, 4, p, p, p, 7, None) == UNSUP
     assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, 42, None) == UNSUP
+    assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, 0x200, None) == UNSUP   # unknown flag
+    assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, 0x102, None) == UNSUP   # removed path, with a flag
+    assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, -1, None) == UNSUP
+    assert lib.ob_linear_ex(None, 0, 64, None, 8, None, None, None, 0, 0x100, None) == OK  # static weights
     # null and alignment
     assert lib.ob_linear(None, 1, 64, p, 4, p, p, p, 0, None) == NULL
     assert lib.ob_linear(p, 1, 64, p, 4, p, p, None, 0, None) == NULL

@@ -15,7 +15,7 @@ from helpers import Guarded, assert_gemm_close, oracle_svid
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5}
+PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5, "auto_static": 0x100, "simt_static": 0x101}
 
 
 @pytest.fixture(scope="module")
@@ -173,7 +173,7 @@ def test_linear_degenerate_sizes(ops):
 
 # ---------------------------------------------------------------- full-size workloads
 
-@pytest.mark.parametrize("path", ["mma_decode", "simt", "i8"])
+@pytest.mark.parametrize("path", ["mma_decode", "simt", "i8", "auto_static"])
 @pytest.mark.parametrize("M", [1, 2, 4, 16])
 def test_decode_workload_full(ops, path, M):
     # OneBit decode GEMV: X M x 4096, W 4096 x 4096 -> 2 MiB packed, a, b from SVID.
@@ -237,7 +237,7 @@ def test_cuda_graph_replay_matches(ops):
 
 
 @pytest.mark.parametrize("M,path", [(1, "auto"), (4, "auto"), (16, "auto"), (40, "auto"), (1, "i8"), (2, "i8"), (3, "i8"),
-                                    (16, "i8")])
+                                    (16, "i8"), (1, "auto_static"), (3, "simt_static"), (16, "auto_static")])
 def test_chained_layers_in_graph(ops, M, path):
     # Eight 512 x 512 layers chained through their outputs (layer i+1 reads layer i's Y),
     # captured in one CUDA graph; calls may launch before their predecessor has finished
