@@ -249,10 +249,12 @@ __device__ __forceinline__ void load_sb_regs(const uint32_t* fr, int lane, SbReg
 __device__ __forceinline__ void tile_sb_regs(const SbRegs& fr, uint4 wg, uint4 wh, int (&acc)[kChains][4]) {
   const uint32_t g4[4] = {wg.x, wg.y, wg.z, wg.w};
   const uint32_t h4[4] = {wh.x, wh.y, wh.z, wh.w};
+  // Position-major order: the four chains take turns, so consecutive MMAs never depend on
+  // each other.
 #pragma unroll
-  for (int p = 0; p < 2; ++p)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int p = 0; p < 2; ++p) {
       const uint32_t g0 = g4[2 * p] >> (2 * i), h0 = h4[2 * p] >> (2 * i);
       const uint32_t g1 = g4[2 * p + 1] >> (2 * i), h1 = h4[2 * p + 1] >> (2 * i);
 #pragma unroll
