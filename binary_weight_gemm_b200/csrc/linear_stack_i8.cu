@@ -258,7 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
     if (s0.layer >= 0 && copier_warp) {
       load_desc(p, s0.layer, &s_desc[cur], lane);
       __syncwarp();
-      if (tid == kCopyThread) fetch_seg(s_desc[cur], s0, wbuf, &wbar);
+      if (tid == kCopyThread) {
+        fetch_seg(s_desc[cur], s0, wbuf, &wbar);
+        const Seg s1 = first_seg(scg, 1);  // the second group's scales (later ones: at the barriers)
+        if (s1.layer >= 0) prefetch_scales(p.L[s1.layer], s1);
+      }
     }
     pending = s0;
   }
@@ -446,7 +450,16 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
     staged = -1;  // the next group's inputs are new
     if (gi + 1 < ng) {
       ++barriers;
-      if (!grid_barrier(p.bar, barriers * (unsigned)G, p.err, &s_ok)) {
+      // While thread 0 waits, the copy thread requests the scale vectors of the group after
+      // the next into L2 (the next group's were requested with its weights, which is late for
+      // the input scale its staging reads first).
+      const auto side = [&]() {
+        if (tid == kCopyThread) {
+          const Seg a = first_seg(scg, gi + 2);
+          if (a.layer >= 0) prefetch_scales(p.L[a.layer], a);
+        }
+      };
+      if (!grid_barrier(p.bar, barriers * (unsigned)G, p.err, &s_ok, side)) {
         // Leave no bulk copy in flight into this CTA's shared memory.
         if (pending.layer >= 0) mbar_wait(&wbar, wphase & 1u, p.err, nullptr);
         return;

@@ -54,8 +54,17 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 // or another CTA aborted.  The wait is bounded: a CTA that gives up records a
 // timeout in the error word and sets the abort word, which makes every other CTA
 // leave at its next barrier.
-__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned target, unsigned* err, int* s_ok) {
+struct NoSideWork {
+  __device__ void operator()() const {}
+};
+
+// `side` runs on every thread but thread 0 while thread 0 waits (work that needs no
+// results of this barrier, e.g. prefetches for later groups).
+template <class Side = NoSideWork>
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, unsigned target, unsigned* err, int* s_ok,
+                                             const Side& side = Side()) {
   __syncthreads();
+  if (threadIdx.x != 0) side();
   if (threadIdx.x == 0) {
     __threadfence();  // this CTA's outputs before its arrival
     atomicAdd(bar, 1u);
