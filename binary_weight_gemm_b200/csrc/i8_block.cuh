@@ -13,19 +13,20 @@
 // (native on sm_100a: e4m3 and 4-bit forms measured three to twenty times slower with
 // operands that change every instruction):
 //
-//  * x' is quantised per token and per staged chunk of k: q = rint(x' sigma) with a
+//  * x' is quantised per token and per super-block of 512 k: q = rint(x' sigma) with a
 //    power-of-two sigma such that |q| <= 2^20, and split into three base-128 limbs
 //    q = l0 + 128 l1 + 16384 l2 (l0, l1 in [0, 128), l2 in [-64, 64]).  Column n = 3 m + l of
 //    the B operand holds limb l of token m.  The rounding is the only approximation (2^-21
-//    of the chunk's largest |x'|).
+//    of the super-block's largest |x'|); one warp stages a (token, super-block) pair on its
+//    own, scale included.
 //  * A (16 rows x 32 k, weights): for bit position j = 2i + c (i = 0..3, c = 0, 1) the
 //    register (w >> 2i) & (0x01010101 << c) of a packed word w holds, in byte i', bit
 //    8i' + j of w at bit c: the u8 value 2^c bit (one shift per word and i, one AND per
 //    four weights).  One MMA takes a single position j from two packed words (a0/a1 from
 //    word 2p, a2/a3 from word 2p+1 of the lane's four) and accumulates into chain (p, c):
 //    four chains, whose sum of acc >> c is the exact integer sum of bit * limb.
-//  * The integer sums are converted and scaled, -2 * 128^l / sigma per column, when a
-//    tile's share of a chunk is done; T is added in the epilogue.
+//  * The integer sums of a (tile, super-block) are converted and scaled, -2 * 128^l / sigma
+//    per column; T is added in the epilogue.
 //
 // Fragment correspondence (PTX ISA, mma.m16n8k32 with 8-bit operands): lane (g, t) holds
 // A rows g and g+8, k-slots 4t + i (a0, a1) and 16 + 4t + i (a2, a3), and B column g,
@@ -66,20 +67,19 @@ __device__ __forceinline__ float pow2(int e) { return __uint_as_float((uint32_t)
 template <int TOK>
 struct Stage {
   uint32_t* frag;  // [ch][p][j][lane][2]
-  float* pmax;     // [ch][TOK]: largest |x'| of a (super-block, token) pair
+  float* fsb;      // [ch][8]: fold factor of each accumulator column for the super-block
   float* tsb;      // [ch][TOK]: sum of x' over the super-block, per token
-  float* fcol;     // [8]: fold factor of each accumulator column for the chunk
   __device__ __forceinline__ uint32_t* frag_at(int s) const { return frag + (size_t)s * kFragWords; }
+  __device__ __forceinline__ const float* fold_at(int s) const { return fsb + (size_t)s * 8; }
   static __host__ __device__ constexpr size_t bytes_per_sb() {
-    return sizeof(uint32_t) * kFragWords + 2 * sizeof(float) * TOK;
+    return sizeof(uint32_t) * kFragWords + sizeof(float) * (8 + TOK);
   }
-  static __host__ __device__ constexpr size_t bytes(int ch) { return bytes_per_sb() * (size_t)ch + 8 * sizeof(float); }
+  static __host__ __device__ constexpr size_t bytes(int ch) { return bytes_per_sb() * (size_t)ch; }
   __device__ static Stage carve(uint8_t* base, int ch) {
     Stage st;
     st.frag = reinterpret_cast<uint32_t*>(base);
-    st.pmax = reinterpret_cast<float*>(base + sizeof(uint32_t) * (size_t)ch * kFragWords);
-    st.tsb = st.pmax + (size_t)ch * TOK;
-    st.fcol = st.tsb + (size_t)ch * TOK;
+    st.fsb = reinterpret_cast<float*>(base + sizeof(uint32_t) * (size_t)ch * kFragWords);
+    st.tsb = st.fsb + (size_t)ch * 8;
     return st;
   }
 };
@@ -122,42 +122,6 @@ __device__ __forceinline__ void stage_values(const StageRaw& raw, float (&v)[4][
   }
 }
 
-// Phase 1 of staging a pair: its largest |x'| and its sum of x' into slot s of the stage.
-template <int TOK>
-__device__ __forceinline__ void stage_measure(const StageRaw& raw, int m, const Stage<TOK>& st, int s, int lane) {
-  float v[4][4];
-  stage_values(raw, v);
-  float amax = 0.f, tpart = 0.f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      amax = fmaxf(amax, fabsf(v[i][jj]));
-      tpart += v[i][jj];
-    }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    tpart += __shfl_xor_sync(0xffffffffu, tpart, o);
-  }
-  if (lane == 0) {
-    st.pmax[s * TOK + m] = amax;
-    st.tsb[s * TOK + m] = tpart;
-  }
-}
-
-// The exponent sg of the chunk's scale sigma = 2^sg for token m (max |x'| sigma < 2^20),
-// from the pair maxima of the chunk's chn super-blocks.  All lanes of a warp call it.
-template <int TOK>
-__device__ __forceinline__ int chunk_exponent(const Stage<TOK>& st, int chn, int m, int lane) {
-  float amax = 0.f;  // lane s takes super-blocks s, s + 32, ...; then a warp-wide maximum
-  for (int s = lane; s < chn; s += 32) amax = fmaxf(amax, st.pmax[s * TOK + m]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127 : 0;
-  return max(-100, min(100, 19 - (e < -126 ? -126 : e)));
-}
-
 // q = rint(y) for |y| < 2^22, by the float magic-number rounding (one FFMA, one integer
 // subtract: round to nearest even, as the FFMA rounds).
 __device__ __forceinline__ int rint_small(float v, float sigma) {
@@ -177,13 +141,29 @@ __device__ __forceinline__ void limb_regs(int q0, int q1, int q2, int q3, uint32
   reg[2] = __byte_perm(__byte_perm(f0, f1, 0x0062), __byte_perm(f2, f3, 0x0062), 0x5410);
 }
 
-// Phase 2: quantise the pair with token m's exponent sg and write its B registers (three
-// limbs each) into slot s.
+// Stage a (token m, super-block s) pair into slot s: the pair's largest |x'| gives its scale
+// sigma = 2^sg (max |x'| sigma < 2^20), its limbs go to the B fragments, its fold factors
+// (-2 * 128^l / sigma for columns 3 m + l; the warp of token 0 also zeroes the unused
+// columns) and its sum of x' to the slot's tables.  All lanes of a warp call it.
 template <int TOK>
-__device__ __forceinline__ void stage_quantise(const StageRaw& raw, int m, int sg, const Stage<TOK>& st, int s,
-                                               int lane) {
+__device__ __forceinline__ void stage_pair(const StageRaw& raw, int m, const Stage<TOK>& st, int s, int lane) {
   float v[4][4];
   stage_values(raw, v);
+  float amax = 0.f, tpart = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      amax = fmaxf(amax, fabsf(v[i][jj]));
+      tpart += v[i][jj];
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    tpart += __shfl_xor_sync(0xffffffffu, tpart, o);
+  }
+  const int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127 : 0;
+  const int sg = max(-100, min(100, 19 - (e < -126 ? -126 : e)));
   const int q = lane >> 1, jh = (lane & 1) * 4;
   const int t = q >> 2, ee = q & 3, p = ee >> 1, half = ee & 1;
   const float sigma = pow2(sg);
@@ -200,6 +180,10 @@ __device__ __forceinline__ void stage_quantise(const StageRaw& raw, int m, int s
       fr[((p * 8 + j) * 32 + 4 * gc + t) * 2 + half] = reg[l];
     }
   }
+  float* f = st.fsb + (size_t)s * 8;
+  if (lane < kLimbs) f[kLimbs * m + lane] = -2.f * pow2(7 * lane - sg);
+  if (m == 0 && lane >= kLimbs * TOK && lane < 8) f[lane] = 0.f;
+  if (lane == 0) st.tsb[s * TOK + m] = tpart;
 }
 
 // Chains per tile: (p, c) with p the word pair and c the parity of the bit position.
@@ -266,17 +250,6 @@ __device__ __forceinline__ void tile_sb_regs(const SbRegs& fr, uint4 wg, uint4 w
 // bit * limb.
 __device__ __forceinline__ int combine(const int (&acc)[kChains][4], int r) {
   return (acc[0][r] + acc[2][r]) + ((acc[1][r] + acc[3][r]) >> 1);
-}
-
-// The fold factors of the chunk's columns: -2 * 128^l / sigma_m for column 3 m + l (0 for
-// unused columns), written by one thread.
-template <int TOK>
-__device__ __forceinline__ void write_fcol(const Stage<TOK>& st, const int (&sg)[TOK]) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const int m = c / kLimbs, l = c % kLimbs;
-    st.fcol[c] = m < TOK ? -2.f * pow2(7 * l - sg[m < TOK ? m : 0]) : 0.f;
-  }
 }
 
 // Packed words of rows g / g+8 of a row tile for a super-block, from global memory: words

@@ -82,7 +82,8 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_i8_kernel(SignGemmArgs g, 
       }
     }
     __syncthreads();  // the previous chunk's stage is no longer read
-    // Staging, phase 1: the pairs (token, super-block) p = warp, warp + 8, warp + 16.
+    // Staging: the pairs (token, super-block) p = warp, warp + 8, warp + 16, each with its own
+    // scale.
     StageRaw raw[kMaxPairs];
 #pragma unroll
     for (int k = 0; k < kMaxPairs; ++k) {
@@ -92,41 +93,35 @@ __global__ void __launch_bounds__(kThreads) sign_gemm_i8_kernel(SignGemmArgs g, 
 #pragma unroll
     for (int k = 0; k < kMaxPairs; ++k) {
       const int p = warp + k * kWarps;
-      if (p < TOK * chn) stage_measure<TOK>(raw[k], p % TOK, st, p / TOK, lane);
+      if (p < TOK * chn) stage_pair<TOK>(raw[k], p % TOK, st, p / TOK, lane);
     }
     __syncthreads();
-    // Phase 2: the chunk's scale per token, then the limbs.
-    int sg[TOK];
-#pragma unroll
-    for (int m = 0; m < TOK; ++m) sg[m] = chunk_exponent<TOK>(st, chn, m, lane);
-#pragma unroll
-    for (int k = 0; k < kMaxPairs; ++k) {
-      const int p = warp + k * kWarps;
-      if (p < TOK * chn) stage_quantise<TOK>(raw[k], p % TOK, sg[p % TOK], st, p / TOK, lane);
-    }
     if (warp == kWarps - 1) {
-      if (lane == 0) write_fcol<TOK>(st, sg);
 #pragma unroll
       for (int m = 0; m < TOK; ++m) {
         const float t = chunk_sum<TOK>(st, chn, m, lane);
         if (lane == 0) tsum[m] += t;
       }
     }
-    __syncthreads();
-    // Multiply: exact int32 sums per bit position over the warp's items, folded once.
-    int acc[kChains][4];
-#pragma unroll
-    for (int j = 0; j < kChains; ++j)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) acc[j][r] = 0;
+    // Multiply: exact int32 sums per (tile, super-block), folded with the super-block's
+    // factors.
+    const int c0 = 2 * tq;
 #pragma unroll
     for (int it = 0; it < kItems; ++it) {
       const int s = warp / kRT + it * kStride;
-      if (s < chn) tile_sb(st.frag_at(s), wg[it], wh[it], acc, lane);
-    }
-    const float f0 = st.fcol[2 * tq], f1 = st.fcol[2 * tq + 1];
+      if (s < chn) {
+        int acc[kChains][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) tot[r] = fmaf((float)combine(acc, r), (r & 1) ? f1 : f0, tot[r]);
+        for (int j = 0; j < kChains; ++j)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) acc[j][r] = 0;
+        tile_sb(st.frag_at(s), wg[it], wh[it], acc, lane);
+        const float* f = st.fold_at(s);
+        const float f0 = f[c0], f1 = f[c0 + 1];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) tot[r] = fmaf((float)combine(acc, r), (r & 1) ? f1 : f0, tot[r]);
+      }
+    }
     // Items past kItems (a chunk longer than kItems * 4 super-blocks) are not possible:
     // chunk_max() <= 24 = kItems * kStride.
   }

@@ -307,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
         if (!(single_chunk && staged == sg.layer)) {
           // Earlier readers of the stage and of tsum are done: the barrier at the top of the
           // segment (first chunk) or the one after the previous chunk's multiply.
-          // Staging, phase 1: the pairs (token, super-block) p = warp, warp + 8, warp + 16.
+          // Staging: the pairs (token, super-block) p = warp, warp + 8, warp + 16, each with
+          // its own scale; then warp 7 sums T while the others start multiplying.
           StageRaw raw[kMaxPairs];
 #pragma unroll
           for (int k = 0; k < kMaxPairs; ++k) {
@@ -317,27 +318,16 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
 #pragma unroll
           for (int k = 0; k < kMaxPairs; ++k) {
             const int pp = warp + k * kWarps;
-            if (pp < TOK * chn) stage_measure<TOK>(raw[k], pp % TOK, st, pp / TOK, lane);
+            if (pp < TOK * chn) stage_pair<TOK>(raw[k], pp % TOK, st, pp / TOK, lane);
           }
           __syncthreads();
-          // Phase 2: the chunk's scale per token, then the limbs.
-          int sgx[TOK];
-#pragma unroll
-          for (int m = 0; m < TOK; ++m) sgx[m] = chunk_exponent<TOK>(st, chn, m, lane);
-#pragma unroll
-          for (int k = 0; k < kMaxPairs; ++k) {
-            const int pp = warp + k * kWarps;
-            if (pp < TOK * chn) stage_quantise<TOK>(raw[k], pp % TOK, sgx[pp % TOK], st, pp / TOK, lane);
-          }
           if (warp == kWarps - 1) {
-            if (lane == 0) write_fcol<TOK>(st, sgx);
 #pragma unroll
             for (int m = 0; m < TOK; ++m) {
               const float t = chunk_sum<TOK>(st, chn, m, lane);
               if (lane == 0) tsum[m] = (sb0 == 0 ? 0.f : tsum[m]) + t;
             }
           }
-          __syncthreads();
           staged = single_chunk ? sg.layer : -1;
         }
         if (sb0 == 0) {  // this segment's weights
@@ -354,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
         if (!s_abort && chn <= kWarps) {
           // At most one super-block per warp (K <= 4096 in one chunk): its fragments stay in
           // registers for all the tiles, and each tile's words are requested one tile ahead.
-          const float f0 = st.fcol[2 * tq], f1 = st.fcol[2 * tq + 1];
           const int s = warp;
+          const float f0 = s < chn ? st.fold_at(s)[2 * tq] : 0.f, f1 = s < chn ? st.fold_at(s)[2 * tq + 1] : 0.f;
           SbRegs fr;
           if (s < chn) load_sb_regs(st.frag_at(s), lane, fr);
           const int64_t w0 = (sb0 + s) * kSbWords + 4 * tq;
@@ -387,25 +377,28 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
             wh = nh;
           }
         } else if (!s_abort) {
-          const float f0 = st.fcol[2 * tq], f1 = st.fcol[2 * tq + 1];
           for (int i = 0; i < sg.nt; ++i) {
-            int acc[kChains][4];
-#pragma unroll
-            for (int j = 0; j < kChains; ++j)
-#pragma unroll
-              for (int r = 0; r < 4; ++r) acc[j][r] = 0;
+            float v[4] = {0.f, 0.f, 0.f, 0.f};
             for (int s = warp; s < chn; s += kWarps) {
+              int acc[kChains][4];
+#pragma unroll
+              for (int j = 0; j < kChains; ++j)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc[j][r] = 0;
               const int64_t w0 = (sb0 + s) * kSbWords + 4 * tq;
               const uint4 wg = smem_words(wbuf, Wd, 16 * i + gq, nrows, w0, L.vec != 0);
               const uint4 wh = smem_words(wbuf, Wd, 16 * i + gq + 8, nrows, w0, L.vec != 0);
               tile_sb(st.frag_at(s), wg, wh, acc, lane);
+              const float* f = st.fold_at(s);
+              const float f0 = f[2 * tq], f1 = f[2 * tq + 1];
+#pragma unroll
+              for (int r = 0; r < 4; ++r) v[r] = fmaf((float)combine(acc, r), (r & 1) ? f1 : f0, v[r]);
             }
             float* dst = red + (size_t)(i * kWarps + warp) * 128;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-              const float v = (float)combine(acc, r) * ((r & 1) ? f1 : f0);
               float* d = dst + r * 32 + lane;
-              *d = sb0 == 0 ? v : *d + v;
+              *d = sb0 == 0 ? v[r] : *d + v[r];
             }
           }
         }
