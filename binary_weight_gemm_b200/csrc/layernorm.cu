@@ -6,7 +6,8 @@
 // affine parameters (the page shows none).
 //
 // A token's N outputs come from many CTAs of the GEMM, so normalisation is a second
-// pass; it reads each row twice (the second read hits L1/L2) and writes it once.
+// pass.  bf16 rows of up to 16384 features are read once into registers and written once;
+// other rows are read twice (the second read hits L1/L2) and written once.
 // One CTA per row.  Statistics: each thread sums y - y0 and (y - y0)^2 in fp32 over
 // its strided elements (y0 = the row's first element, so a large mean does not
 // cancel the variance away), the CTA combines the partial sums in fp64.
@@ -36,6 +37,25 @@ __device__ __forceinline__ void store_z(void* row, int64_t j, float z) {
     static_cast<__nv_bfloat16*>(row)[j] = __float2bfloat16_rn(z);
   else
     static_cast<float*>(row)[j] = z;
+}
+
+// Sums of two doubles over the CTA in one reduction; every thread gets the results.
+__device__ __forceinline__ double2 block_sum2(double a, double b, double2* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = make_double2(a, b);
+  __syncthreads();
+  double2 t = make_double2(0.0, 0.0);
+#pragma unroll
+  for (int w = 0; w < kLnThreads / 32; ++w) {
+    t.x += red[w].x;
+    t.y += red[w].y;
+  }
+  return t;
 }
 
 // Sum of a double over the CTA; every thread gets the result.
@@ -108,6 +128,56 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_rows_kernel(void* Y, int
   }
 }
 
+// bf16 rows with N % 8 == 0, 16-byte aligned, and N / 8 <= 256 V: one pass.  Each thread
+// keeps its V 16-byte pieces of the row in registers, so Y is read once and written once.
+template <int V>
+__global__ void __launch_bounds__(kLnThreads) layernorm_rows_reg_kernel(void* Y, int64_t N, int64_t ld, float eps) {
+  __shared__ double2 red[kLnThreads / 32];
+  pdl_wait();  // Y is written by the previous grid
+  pdl_launch_dependents();
+  uint4* r4 = reinterpret_cast<uint4*>(static_cast<char*>(Y) + (int64_t)blockIdx.x * ld * 2);
+  const int64_t n8 = N / 8;
+  const float y0 = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(r4)[0] << 16);
+  uint4 v[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int64_t idx = threadIdx.x + (int64_t)i * kLnThreads;
+    v[i] = idx < n8 ? r4[idx] : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    if (threadIdx.x + (int64_t)i * kLnThreads >= n8) continue;
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = __uint_as_float(w[e] << 16) - y0, hi = __uint_as_float(w[e] & 0xFFFF0000u) - y0;
+      s1 += lo + hi;
+      s2 = fmaf(lo, lo, fmaf(hi, hi, s2));
+    }
+  }
+  const double2 S = block_sum2((double)s1, (double)s2, red);
+  const double S1 = S.x, S2 = S.y;
+  const double dmean = S1 / (double)N;  // mean - y0
+  const double var = fmax(S2 / (double)N - dmean * dmean, 0.0);
+  const float mean = (float)((double)y0 + dmean);
+  const float rstd = (float)(1.0 / sqrt(var + (double)eps));
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int64_t idx = threadIdx.x + (int64_t)i * kLnThreads;
+    if (idx >= n8) continue;
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = (__uint_as_float(w[e] << 16) - mean) * rstd;
+      const float hi = (__uint_as_float(w[e] & 0xFFFF0000u) - mean) * rstd;
+      o[e] = pack_bf16x2(lo, hi);
+    }
+    r4[idx] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_layernorm_rows(void* Y, int64_t M, int64_t N, int64_t ld, int y_dtype, float eps,
@@ -123,8 +193,20 @@ cudaError_t launch_layernorm_rows(void* Y, int64_t M, int64_t N, int64_t ld, int
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = c.pdl ? 1 : 0;
-  cudaError_t e = y_dtype == OB_OUT_F32 ? cudaLaunchKernelEx(&cfg, layernorm_rows_kernel<false>, Y, N, ld, eps)
-                                        : cudaLaunchKernelEx(&cfg, layernorm_rows_kernel<true>, Y, N, ld, eps);
+  // bf16 rows that fit 8 pieces of 16 bytes per thread (N <= 16384) and allow 16-byte access
+  // take the one-pass kernel.
+  const bool reg = y_dtype == OB_OUT_BF16 && N % 8 == 0 && ld % 8 == 0 &&
+                   (reinterpret_cast<uintptr_t>(Y) & 15) == 0 && N / 8 <= 8 * kLnThreads;
+  const int64_t per = (N / 8 + kLnThreads - 1) / kLnThreads;  // 16-byte pieces per thread
+  cudaError_t e;
+  if (reg)
+    e = per <= 1   ? cudaLaunchKernelEx(&cfg, layernorm_rows_reg_kernel<1>, Y, N, ld, eps)
+        : per <= 2 ? cudaLaunchKernelEx(&cfg, layernorm_rows_reg_kernel<2>, Y, N, ld, eps)
+        : per <= 4 ? cudaLaunchKernelEx(&cfg, layernorm_rows_reg_kernel<4>, Y, N, ld, eps)
+                   : cudaLaunchKernelEx(&cfg, layernorm_rows_reg_kernel<8>, Y, N, ld, eps);
+  else
+    e = y_dtype == OB_OUT_F32 ? cudaLaunchKernelEx(&cfg, layernorm_rows_kernel<false>, Y, N, ld, eps)
+                              : cudaLaunchKernelEx(&cfg, layernorm_rows_kernel<true>, Y, N, ld, eps);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
