@@ -959,6 +959,15 @@ def run_extra(ops, dev, stream, peaks):
                         "tflops_equiv": 2 * M * 4096 * 4096 / t / 1e12, "tflops_alg": fl / t / 1e12,
                         "hbm_gbs": byts / t / 1e9, "frac_hbm": byts / t / 1e9 / peaks["hbm_gbs"],
                         "frac_bf16_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
+            if M == 1 and r == 2048:
+                # The two products as two per-call kernels (CUDA-core table kernel at one token),
+                # with static weights, beside the one-launch form AUTO takes.
+                t2 = timer(lambda i: ops.dbf_linear(X, pool[i % nset][0], vec["m"], pool[i % nset][1], vec["a"],
+                                                    vec["b"], out=Y, workspace=ws, stream=stream,
+                                                    path=ops.OB_PATH_SIMT | ops.OB_FLAG_STATIC_WEIGHTS), stream,
+                           max(50, 2 * nset))
+                out["dbf_M1_two_kernels_static"] = {"us_per_call": t2 * 1e6, "hbm_gbs": byts / t2 / 1e9,
+                                                    "frac_hbm": byts / t2 / 1e9 / peaks["hbm_gbs"]}
             del pool
     return out
 

@@ -338,6 +338,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
         launch_sign_stack(two, 2, M, bar, c, M <= kStackI8MaxM ? OB_PATH_I8 : OB_PATH_MMA_DECODE));
   }
   SignGemmArgs g1{static_cast<const uint16_t*>(X), M, K, SB_packed, r, b, m, T, r, OB_OUT_BF16};
+  g1.static_w = static_w;  // S_B, b, m
   // Few output tiles (small M x r): split the first product over K into fp32 partial
   // sums after T in the workspace, when the workspace holds them.
   const bool tc1 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > kDecodeMaxM && K <= sign_gemm_tc_max_k());
@@ -352,6 +353,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   }
   if (st != OB_OK) return st;
   SignGemmArgs g2{T, M, r, SA_packed, N, nullptr, a, Y, N, y_dtype};
+  g2.static_w = static_w;  // S_A, a (T is the previous kernel's output: read after the wait)
   // The second product (K = r) splits the same way when the region after T also holds
   // its partial sums (the first product's are consumed before it runs), unless the
   // CTA-pair kernel takes it and r < 4096: measured at M = 512 on B200, r = 2048

@@ -9,7 +9,7 @@ from helpers import Guarded, assert_gemm_close
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5, "auto": 0}
+PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5, "auto": 0, "simt_static": 0x101, "mma_static": 0x104}
 
 
 @pytest.fixture(scope="module")
@@ -45,7 +45,7 @@ def _ref(x, f):
     return oracle.dbf_linear(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"])
 
 
-@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "i8", "auto"])
+@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "i8", "auto", "simt_static", "mma_static"])
 @pytest.mark.parametrize("M,N,r,K", [(1, 128, 32, 64), (4, 256, 96, 256), (7, 200, 160, 96), (33, 130, 64, 128),
                                      (260, 256, 128, 320)])
 def test_dbf_small_shapes(ops, path, M, N, r, K):
