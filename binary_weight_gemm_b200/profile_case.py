@@ -3,6 +3,7 @@
     python -m binary_weight_gemm_b200.profile_case decode --m 16 --reps 40 [--static]
     python -m binary_weight_gemm_b200.profile_case prefill --reps 6
     python -m binary_weight_gemm_b200.profile_case dbf --m 512 --reps 6
+    python -m binary_weight_gemm_b200.profile_case dbf --m 1 --reps 20 --static [--path stack]
     python -m binary_weight_gemm_b200.profile_case stack --m 1 --blocks 8 --reps 5
     python -m binary_weight_gemm_b200.profile_case stack --m 1 --chain 128 --reps 5 --path i8
 
@@ -46,14 +47,16 @@ def main(argv=None) -> None:
     ap.add_argument("--reps", type=int, default=6)
     ap.add_argument("--blocks", type=int, default=8, help="stack: 7B-shaped blocks")
     ap.add_argument("--chain", type=int, default=0, help="stack: chained 1024 -> 1024 layers instead")
-    ap.add_argument("--path", choices=("auto", "mma", "i8"), default="auto",
-                    help="stack / decode: kernel form (AUTO, the bf16 warp MMA, or the int8 form)")
+    ap.add_argument("--path", choices=("auto", "mma", "i8", "stack"), default="auto",
+                    help="stack / decode / dbf: kernel form (AUTO, the bf16 warp MMA, the int8 form; dbf also "
+                         "'stack': both products in one persistent launch)")
     ap.add_argument("--static", action="store_true",
-                    help="decode: OR OB_FLAG_STATIC_WEIGHTS into the path (as the benchmark's decode calls do)")
+                    help="decode / dbf: OR OB_FLAG_STATIC_WEIGHTS into the path (as the benchmark's decode calls do)")
     args = ap.parse_args(argv)
     dev = torch.device("cuda", 0)
     torch.cuda.init()
-    path = {"auto": ops.OB_PATH_AUTO, "mma": ops.OB_PATH_MMA_DECODE, "i8": ops.OB_PATH_I8}[args.path]
+    path = {"auto": ops.OB_PATH_AUTO, "mma": ops.OB_PATH_MMA_DECODE, "i8": ops.OB_PATH_I8,
+            "stack": ops.OB_PATH_STACK}[args.path]
     lin_path = path | (ops.OB_FLAG_STATIC_WEIGHTS if args.static else 0)
 
     if args.case in ("decode", "prefill"):
@@ -119,7 +122,7 @@ def main(argv=None) -> None:
 
         def call(i):
             X, SBq, SAq, Y = sets[i % n_sets]
-            ops.dbf_linear(X, SBq, mvec, SAq, a, b, out=Y, workspace=ws)
+            ops.dbf_linear(X, SBq, mvec, SAq, a, b, out=Y, workspace=ws, path=lin_path)
 
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

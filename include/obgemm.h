@@ -89,9 +89,11 @@ typedef enum ob_path {
   OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA); K <= 32768; a
                               2-CTA (cta_group::2) tile where bf16 Y, M >= 512, N >= 256, K <= 16384 */
   OB_PATH_MMA_DECODE = 4,  /* bf16 warp-level MMA, signs unpacked in registers, M <= 16 per pass */
-  OB_PATH_I8 = 5           /* int8 warp-level MMA (u8 x s8 -> s32): each packed word becomes eight operand
+  OB_PATH_I8 = 5,          /* int8 warp-level MMA (u8 x s8 -> s32): each packed word becomes eight operand
                               registers with one AND each, activations quantised per token to 21 bits in
                               three 7-bit limbs, exact integer sums; M <= 2 per pass */
+  OB_PATH_STACK = 6        /* dbf_linear_ex only, M <= 16: both sign products in one persistent launch of
+                              the layer-stack kernel, a grid barrier between them */
 } ob_path;
 
 /* Flag OR-ed into the path argument of ob_linear_ex (and ob_linear_ln): the caller
@@ -254,12 +256,12 @@ OB_API ob_status ob_linear_stack_ex(const ob_layer* layers, int n_layers, int64_
 
 /*
  * Bytes of device workspace dbf_linear uses: the M x r bf16 intermediate T, 256 bytes
- * after it (the grid-barrier word of the one-launch decode chain) and, when the first
+ * after it (the grid-barrier word of the OB_PATH_STACK form) and, when the first
  * product runs on the tcgen05 GEMM with fewer output tiles than half the SMs of the
  * current device (e.g. M = 512, r = 2048), fp32 partial sums for splitting it over K
  * (up to 8 x M x r x 4 bytes).  dbf_linear accepts any workspace of at least T's size
  * (M x r x 2 rounded up to 256 bytes); a smaller one than this function returns runs the
- * decode chain as two launches, and the first product without the split.
+ * first product without the split (and rejects OB_PATH_STACK with OB_ERR_WORKSPACE).
  */
 OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
 
@@ -276,10 +278,11 @@ OB_API size_t dbf_workspace_size(int64_t M, int64_t r);
  *   workspace  device, at least dbf_workspace_size(M, r) bytes; holds the
  *              intermediate T = ((X ⊙ b^T) S_B^T) ⊙ m^T between the two sign
  *              products (it stays in L2 at the workload sizes).
- * K % 32 == 0, r % 32 == 0.  Asynchronous.  M <= 16 (decode): both products run in
- * one persistent launch (the layer-stack kernels with a grid barrier between the two
- * products; int8 form for M <= 2), so T never leaves the chip's L2 between them; larger
- * M: two tcgen05 GEMMs.
+ * K % 32 == 0, r % 32 == 0.  Asynchronous.  M <= 16 (decode): the two products are two
+ * decode kernels chained by programmatic dependent launch; T (M x r bf16, a few KB) is
+ * written to L2 and read back from it by the second.  Larger M: two tcgen05 GEMMs, the
+ * first split over K when it has few output tiles.  dbf_linear_ex with OB_PATH_STACK runs
+ * both products in one persistent launch instead (measured slower at decode sizes).
  */
 OB_API ob_status dbf_linear(const void* X, int64_t M, int64_t K,
                      const uint32_t* SB_packed, int64_t r, const float* m,

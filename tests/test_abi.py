@@ -79,6 +79,11 @@ def test_host_argument_checks_without_gpu(lib):
     assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, 0x102, None) == UNSUP   # removed path, with a flag
     assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, -1, None) == UNSUP
     assert lib.ob_linear_ex(None, 0, 64, None, 8, None, None, None, 0, 0x100, None) == OK  # static weights
+    assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, 6, None) == UNSUP   # the one-launch DBF form
+    # dbf_linear_ex: the one-launch form only at decode sizes; unknown flags rejected
+    assert lib.dbf_linear_ex(p, 17, 64, p, 32, p, p, 4, p, p, p, 0, p, 1 << 20, 6, None) == UNSUP
+    assert lib.dbf_linear_ex(p, 1, 64, p, 32, p, p, 4, p, p, p, 0, p, 1 << 20, 0x400, None) == UNSUP
+    assert lib.dbf_linear_ex(p, 1, 64, p, 32, p, p, 4, p, p, p, 0, p, 1 << 20, 7, None) == UNSUP
     # null and alignment
     assert lib.ob_linear(None, 1, 64, p, 4, p, p, p, 0, None) == NULL
     assert lib.ob_linear(p, 1, 64, p, 4, p, p, None, 0, None) == NULL

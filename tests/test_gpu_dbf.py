@@ -9,7 +9,8 @@ from helpers import Guarded, assert_gemm_close
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5, "auto": 0, "simt_static": 0x101, "mma_static": 0x104}
+PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5, "auto": 0, "stack": 6, "simt_static": 0x101,
+         "mma_static": 0x104, "auto_static": 0x100}
 
 
 @pytest.fixture(scope="module")
@@ -45,22 +46,28 @@ def _ref(x, f):
     return oracle.dbf_linear(x, f["S_A"], f["S_B"], f["a"], f["m"], f["b"])
 
 
-@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "i8", "auto", "simt_static", "mma_static"])
+@pytest.mark.parametrize("path", ["simt", "tc", "mma_decode", "i8", "auto", "stack", "simt_static", "mma_static"])
 @pytest.mark.parametrize("M,N,r,K", [(1, 128, 32, 64), (4, 256, 96, 256), (7, 200, 160, 96), (33, 130, 64, 128),
                                      (260, 256, 128, 320)])
 def test_dbf_small_shapes(ops, path, M, N, r, K):
     f = synth.dbf_factors(M + N + r + K, N, r, K)
     xb, x = synth.activations(M + N, M, K)
+    if path == "stack" and M > 16:  # the one-launch form is for decode sizes only
+        from binary_weight_gemm_b200._lib import ObError
+        with pytest.raises(ObError):
+            _run(ops, xb, f, PATHS[path])
+        return
     assert_gemm_close(_run(ops, xb, f, PATHS[path]), _ref(x, f), what=f"dbf {path} {M},{N},{r},{K}")
 
 
-@pytest.mark.parametrize("M", [1, 2, 16, 512])
-def test_dbf_workload_full(ops, M):
+@pytest.mark.parametrize("M,path", [(1, "auto"), (2, "auto"), (16, "auto"), (512, "auto"), (1, "auto_static"),
+                                    (16, "auto_static"), (1, "stack"), (2, "stack"), (16, "stack")])
+def test_dbf_workload_full(ops, M, path):
     # DBF: K = N = 4096, r = 2048; S_A, S_B random +/-1; a, m, b ~ |N(0,1)|*0.02+1e-3.
     f = synth.dbf_factors(3, 4096, 2048, 4096)
     xb, x = synth.activations(3, M, 4096)
-    Y = _run(ops, xb, f, PATHS["auto"])
-    assert_gemm_close(Y, _ref(x, f), what=f"dbf workload M={M}")
+    Y = _run(ops, xb, f, PATHS[path])
+    assert_gemm_close(Y, _ref(x, f), what=f"dbf workload M={M} {path}")
 
 
 # Middle dimensions for about 0.5, 1.5, 1.8 and 2.3 bits per weight at K = N = 4096
@@ -77,8 +84,8 @@ def test_dbf_general_r(ops, r, M):
 
 @pytest.mark.parametrize("M", [1, 4])
 def test_dbf_decode_with_the_smallest_workspace(ops, M):
-    # A workspace that holds only T (no room for the one-launch chain's barrier word) runs
-    # the two products as two launches; both give the oracle's result.
+    # A workspace that holds only T is enough for AUTO (two launches); the one-launch form
+    # needs the barrier word after T and rejects it.
     f = synth.dbf_factors(14 + M, 512, 256, 384)
     xb, x = synth.activations(14, M, 384)
     SB = ops.ob_pack_signs(_cuda(f["S_B"].astype(np.float32)))
@@ -91,6 +98,10 @@ def test_dbf_decode_with_the_smallest_workspace(ops, M):
         torch.cuda.synchronize()
         assert ops.ob_last_device_error() == 0
         assert_gemm_close(Y, _ref(x, f), what=f"dbf M={M} workspace {ws_bytes}")
+    from binary_weight_gemm_b200._lib import ObError
+    with pytest.raises(ObError):
+        ops.dbf_linear(X, SB, _cuda(f["m"]), SA, _cuda(f["a"]), _cuda(f["b"]),
+                       workspace=torch.zeros(t_bytes, dtype=torch.uint8, device="cuda"), path=ops.OB_PATH_STACK)
 
 
 def test_dbf_fp32_output(ops):
