@@ -666,7 +666,8 @@ def run_stack(args, world, rank, local):
     stream = torch.cuda.Stream(device=dev)
     peaks = load_peaks()
     blocks = args.blocks
-    ms_list = (1, 16)
+    ms_list = (1, 2, 16)
+    lin_path = ops.OB_PATH_AUTO | ops.OB_FLAG_STATIC_WEIGHTS  # the weights are written once, before timing
     # One seeded matrix per shape, packed and SVID'd by the library, cloned into every block.
     base = {}
     for K, N in sorted(set(STACK_SHAPES.values())):
@@ -690,14 +691,14 @@ def run_stack(args, world, rank, local):
         for L in layers:
             for name in ("q", "k", "v"):
                 P, a, b = L[name]
-                ops.ob_linear(x, P, a, b, out=buf[name], stream=s)
+                ops.ob_linear(x, P, a, b, out=buf[name], stream=s, path=lin_path)
             P, a, b = L["o"]
-            ops.ob_linear(buf["q"], P, a, b, out=buf["o"], stream=s)
+            ops.ob_linear(buf["q"], P, a, b, out=buf["o"], stream=s, path=lin_path)
             for name in ("gate", "up"):
                 P, a, b = L[name]
-                ops.ob_linear(buf["o"], P, a, b, out=buf[name], stream=s)
+                ops.ob_linear(buf["o"], P, a, b, out=buf[name], stream=s, path=lin_path)
             P, a, b = L["down"]
-            ops.ob_linear(buf["gate"], P, a, b, out=buf["down"], stream=s)
+            ops.ob_linear(buf["gate"], P, a, b, out=buf["down"], stream=s, path=lin_path)
             x = buf["down"]
 
     def spec(m):
@@ -780,9 +781,10 @@ def run_stack(args, world, rank, local):
                        "layers_per_token": calls, "weights_mb": wbytes / 1e6,
                        "l2": f"inputs larger than L2: {blocks * 7} distinct weight buffers ({wbytes / 1e6:.0f} MB)",
                        "graph": "one CUDA graph per token and M holding one ob_linear_stack (persistent, "
-                                "grid barriers between dependent layers; AUTO: int8 form at M=1, bf16 warp-MMA "
-                                "form at M=16; persistent_bf16mma_M1 forces the bf16 form); per_call_* times one ob_linear "
-                                "per layer in a graph with programmatic dependent launch",
+                                "grid barriers between dependent layers; AUTO: int8 form at M=1 and 2, bf16 "
+                                "warp-MMA form at M=16; persistent_bf16mma_M1 forces the bf16 form); per_call_* "
+                                "times one ob_linear per layer (AUTO | OB_FLAG_STATIC_WEIGHTS) in a graph with "
+                                "programmatic dependent launch",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "per_m": per_m,
             "gpu_launches": args.steps * len(ms_list), "clocks": clocks, "cpu_baseline": None,
