@@ -166,13 +166,12 @@ def load_peaks() -> dict:
 
 
 def prefill_kernel_name() -> str:
-    """The tcgen05 GEMM the prefill workload runs: the CTA-pair kernel unless OB_TC2=0."""
-    return "sign_gemm_tc_kernel" if os.environ.get("OB_TC2", "1")[:1] in ("0", "n", "N", "f", "F") \
-        else "sign_gemm_tc2_kernel"
+    """The tcgen05 GEMM AUTO runs on the prefill workload (bf16 Y, M >= 512): the CTA-pair kernel."""
+    return "sign_gemm_tc2_kernel"
 
 
 def prefill_kernel_source():
-    return ("linear_tc.cu",) if prefill_kernel_name() == "sign_gemm_tc_kernel" else ("linear_tc2.cu",)
+    return ("linear_tc2.cu",)
 
 
 def ncu_traffic(kernel_file: str, key: str):

@@ -18,6 +18,7 @@ STATUS_NAMES = {
 }
 OB_OUT_BF16, OB_OUT_F32 = 0, 1
 OB_PATH_AUTO, OB_PATH_SIMT, OB_PATH_TC, OB_PATH_MMA_DECODE, OB_PATH_I8 = 0, 1, 3, 4, 5
+OB_PATH_TC1 = 7  # the one-CTA tcgen05 GEMM even where the CTA pair applies
 OB_PATH_STACK = 6  # dbf_linear only: both products in one persistent launch (M <= 16)
 OB_FLAG_STATIC_WEIGHTS = 0x100  # OR into path: W_packed, a, b not written by the previous kernel
 

@@ -99,6 +99,7 @@ ob_status run_sign_gemm(const SignGemmArgs& g_in, int path, const LaunchCtx& c) 
       // 1260 vs 1170 TFLOP/s for the one-CTA kernel at the prefill workload on B200.
       e = sign_gemm_tc2_supported(g) ? launch_sign_gemm_tc2(g, c) : launch_sign_gemm_tc(g, c);
       break;
+    case OB_PATH_TC1: e = launch_sign_gemm_tc(g, c); break;
     default: return OB_ERR_UNSUPPORTED;
   }
   return status_of(e);
@@ -205,7 +206,7 @@ ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
   if (path < 0 || (path & ~0xFF & ~OB_FLAG_STATIC_WEIGHTS) != 0) return OB_ERR_UNSUPPORTED;
   const int static_w = (path & OB_FLAG_STATIC_WEIGHTS) ? 1 : 0;
   path &= 0xFF;
-  if (path > OB_PATH_I8 || path == 2) return OB_ERR_UNSUPPORTED;
+  if (path > OB_PATH_TC1 || path == 2 || path == OB_PATH_STACK) return OB_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return OB_OK;
   if (!Y || !a) return OB_ERR_NULL;
   if (K > 0 && (!X || !W_packed || !b)) return OB_ERR_NULL;

@@ -15,7 +15,7 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import (OB_FLAG_STATIC_WEIGHTS, OB_PATH_STACK, OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_I8, OB_PATH_MMA_DECODE, OB_PATH_SIMT,  # noqa: F401
+from ._lib import (OB_FLAG_STATIC_WEIGHTS, OB_PATH_STACK, OB_PATH_TC1, OB_OUT_BF16, OB_OUT_F32, OB_PATH_AUTO, OB_PATH_I8, OB_PATH_MMA_DECODE, OB_PATH_SIMT,  # noqa: F401
                    OB_PATH_TC, ObError)
 
 

@@ -87,13 +87,16 @@ typedef enum ob_path {
   OB_PATH_AUTO = 0,        /* M == 1: OB_PATH_SIMT; M <= 16 or K > 32768: OB_PATH_MMA_DECODE; else OB_PATH_TC */
   OB_PATH_SIMT = 1,        /* CUDA-core mat-vec: one token by table lookup, more tokens by select/add */
   OB_PATH_TC = 3,          /* tcgen05 tiled GEMM for large M (activations by TMA); K <= 32768; a
-                              2-CTA (cta_group::2) tile where bf16 Y, M >= 512, N >= 256, K <= 16384 */
+                              2-CTA (cta_group::2) tile where bf16 Y, M >= 512, N >= 256, K <= 16384,
+                              else one CTA per tile */
   OB_PATH_MMA_DECODE = 4,  /* bf16 warp-level MMA, signs unpacked in registers, M <= 16 per pass */
   OB_PATH_I8 = 5,          /* int8 warp-level MMA (u8 x s8 -> s32): each packed word becomes eight operand
                               registers with one AND each, activations quantised per token to 21 bits in
                               three 7-bit limbs, exact integer sums; M <= 2 per pass */
-  OB_PATH_STACK = 6        /* dbf_linear_ex only, M <= 16: both sign products in one persistent launch of
+  OB_PATH_STACK = 6,       /* dbf_linear_ex only, M <= 16: both sign products in one persistent launch of
                               the layer-stack kernel, a grid barrier between them */
+  OB_PATH_TC1 = 7          /* ob_linear_ex / ob_linear_ln only: the one-CTA tcgen05 GEMM even where
+                              OB_PATH_TC would take the CTA pair (tests, measurement); K <= 32768 */
 } ob_path;
 
 /* Flag OR-ed into the path argument of ob_linear_ex (and ob_linear_ln): the caller
@@ -169,7 +172,7 @@ OB_API ob_status ob_svid_rank1(const float* W, int64_t N, int64_t K,
  *   Y         device, M x N, bf16 or fp32 by y_dtype.
  * K % 32 == 0.  Accumulates in fp32.  Asynchronous.  OB_PATH_AUTO picks the
  * table-driven CUDA-core kernel for M == 1, the warp-level MMA decode kernel for
- * M <= 16 (OB_DECODE_MAX_M) and the tiled tcgen05 GEMM above.
+ * M <= 16 (and for K > 32768) and the tiled tcgen05 GEMM above.
  */
 OB_API ob_status ob_linear(const void* X, int64_t M, int64_t K,
                     const uint32_t* W_packed, int64_t N,

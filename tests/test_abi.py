@@ -80,6 +80,9 @@ def test_host_argument_checks_without_gpu(lib):
     assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, -1, None) == UNSUP
     assert lib.ob_linear_ex(None, 0, 64, None, 8, None, None, None, 0, 0x100, None) == OK  # static weights
     assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, 6, None) == UNSUP   # the one-launch DBF form
+    assert lib.ob_linear_ex(p, 1, 64, p, 4, p, p, p, 0, 8, None) == UNSUP
+    assert lib.ob_linear_ex(None, 0, 64, None, 8, None, None, None, 0, 7, None) == OK  # the one-CTA tcgen05 GEMM
+    assert lib.dbf_linear_ex(p, 1, 64, p, 32, p, p, 4, p, p, p, 0, p, 1 << 20, 7, None) == UNSUP
     # dbf_linear_ex: the one-launch form only at decode sizes; unknown flags rejected
     assert lib.dbf_linear_ex(p, 17, 64, p, 32, p, p, 4, p, p, p, 0, p, 1 << 20, 6, None) == UNSUP
     assert lib.dbf_linear_ex(p, 1, 64, p, 32, p, p, 4, p, p, p, 0, p, 1 << 20, 0x400, None) == UNSUP

@@ -15,7 +15,7 @@ from helpers import Guarded, assert_gemm_close, oracle_svid
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5, "auto_static": 0x100, "simt_static": 0x101}
+PATHS = {"simt": 1, "tc": 3, "mma_decode": 4, "i8": 5, "tc1": 7, "auto_static": 0x100, "simt_static": 0x101}
 
 
 @pytest.fixture(scope="module")
@@ -153,8 +153,9 @@ def test_tc_path_rejects_k_beyond_limit(ops):
     K = 32768 + 32
     X = torch.zeros((32, K), dtype=torch.bfloat16, device="cuda")
     P = torch.zeros((128, K // 32), dtype=torch.int32, device="cuda")
-    with pytest.raises(ObError):
-        ops.ob_linear(X, P, torch.ones(128, device="cuda"), torch.ones(K, device="cuda"), path=PATHS["tc"])
+    for path in ("tc", "tc1"):
+        with pytest.raises(ObError):
+            ops.ob_linear(X, P, torch.ones(128, device="cuda"), torch.ones(K, device="cuda"), path=PATHS[path])
 
 
 def test_linear_degenerate_sizes(ops):
@@ -194,10 +195,11 @@ def test_prefill_workload_full_every_element(ops):
 
 
 def test_prefill_one_cta_kernel_sampled_rows(ops):
-    # The one-CTA tcgen05 kernel on the prefill workload; oracle on 64 sampled token rows.
+    # The one-CTA tcgen05 kernel (forced: AUTO takes the CTA pair here) on the prefill
+    # workload; oracle on 64 sampled token rows.
     W, a, b, _ = oracle_svid(2, 11008, 4096)
     xb, x = synth.activations(2, 2048, 4096)
-    Y = _run(ops, xb, W, a, b, PATHS["tc"])
+    Y = _run(ops, xb, W, a, b, PATHS["tc1"])
     rows = np.random.default_rng(0).choice(2048, 64, replace=False)
     rows[:2] = [0, 2047]
     assert_gemm_close(Y[torch.from_numpy(rows).cuda()], _ref(x[rows], W, a, b), what="prefill rows")

@@ -1,13 +1,11 @@
 """GPU parity of the CTA-pair tcgen05 GEMM (linear_tc2.cu) against the fp64 oracle.
 
 OB_PATH_TC (and AUTO above 16 tokens) with bf16 output, M >= 512 and N >= 256 runs
-the pair kernel (OB_TC2=0 selects the one-CTA kernel); these shapes exercise its
+the pair kernel (OB_PATH_TC1 forces the one-CTA kernel); these shapes exercise its
 ragged tiles: N not a multiple of 256
 (a pair whose second CTA has no valid rows), M not a multiple of 256, K with a
 partial 128-k stage.
 """
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -25,13 +23,7 @@ def ops():
     build.build()
     from binary_weight_gemm_b200 import ops as _ops
     torch.cuda.init()
-    old = os.environ.get("OB_TC2")
-    os.environ["OB_TC2"] = "1"
-    yield _ops
-    if old is None:
-        del os.environ["OB_TC2"]
-    else:
-        os.environ["OB_TC2"] = old
+    return _ops
 
 
 def _cuda(x):
@@ -57,8 +49,7 @@ def test_tc2_shapes(ops, M, N, K):
 
 
 def test_tc2_matches_one_cta_kernel(ops):
-    # The same problem on the pair kernel and on the one-CTA kernel (OB_TC2=0).
-    assert os.environ.get("OB_TC2") == "1"
+    # The same problem on the pair kernel (OB_PATH_TC) and on the one-CTA kernel (OB_PATH_TC1).
     M, N, K = 1024, 768, 2048
     W = synth.weights(77, N, K)
     a, b, _ = oracle.svid_rank1(W)
@@ -67,12 +58,7 @@ def test_tc2_matches_one_cta_kernel(ops):
     X = _cuda(xb.view(np.int16)).view(torch.bfloat16)
     A, B = _cuda(a.astype(np.float32)), _cuda(b.astype(np.float32))
     Y2 = ops.ob_linear(X, P, A, B, path=ops.OB_PATH_TC)
-    old = os.environ.get("OB_TC2")
-    os.environ["OB_TC2"] = "0"
-    try:
-        Y1 = ops.ob_linear(X, P, A, B, path=ops.OB_PATH_TC)
-    finally:
-        os.environ["OB_TC2"] = old
+    Y1 = ops.ob_linear(X, P, A, B, path=ops.OB_PATH_TC1)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
     assert_gemm_close(Y2, Y1.double().cpu().numpy(), what="pair vs one-CTA")
