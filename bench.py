@@ -835,8 +835,11 @@ def run_sweep(args, world, rank, local):
             else:
                 nset = max(2, -(-2 * 126 * 2**20 // (2 * M * (K + N))))
                 sets = [(X.clone(), torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for _ in range(nset)]
+                # ob_linear_ws: few-tile problems split over K through this workspace.
+                wsb = ops.ob_linear_workspace_size(M, N, K)
+                ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
                 t = _time_calls(lambda i: ops.ob_linear(sets[i % nset][0], P, a, b, out=sets[i % nset][1],
-                                                        stream=stream), stream, max(10, 3 * nset))
+                                                        stream=stream, workspace=ws), stream, max(10, 3 * nset))
                 del sets
             fl = 2 * M * N * K
             rows[f"{K}x{N}_M{M}"] = {"us_per_call": t * 1e6, "hbm_gbs": call_bytes / t / 1e9,
@@ -851,7 +854,9 @@ def run_sweep(args, world, rank, local):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "onebit_sweep_7b_outliers", "shapes_KxN": [list(x) for x in SWEEP_SHAPES],
                        "M": list(SWEEP_MS), "outliers": "6 channels x60",
-                       "l2": "M<=16: weight pool > 3x L2 in one CUDA graph; M>=256: rotating sets > L2"},
+                       "l2": "M<=16: weight pool > 3x L2 in one CUDA graph; M>=256: rotating sets > L2",
+                       "api": "ob_linear (AUTO); M>=256 with the workspace of ob_linear_workspace_size (split over K "
+                              "where few output tiles)"},
             "per_case": rows, "peak_source": peaks["source"], "gpu_launches": None, "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)

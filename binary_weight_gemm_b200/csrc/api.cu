@@ -198,8 +198,22 @@ ob_status ob_svid_rank1(const float* W, int64_t N, int64_t K, float* a, float* b
   return run_svid(W, N, K, a, b, sigma1, max_iters, tol, iters_out, workspace, c);
 }
 
-ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,
-                       const float* b, void* Y, int y_dtype, int path, void* stream) {
+int sms_for_sizing() {
+  DeviceInfo d;
+  return current_device(&d) == OB_OK && d.num_sms > 0 ? d.num_sms : 148;  // B200 when no device
+}
+
+// K slices for a problem that runs on the one-CTA tcgen05 GEMM with few output tiles (1: no
+// split).  The slices' partial sums are summed by a kernel that writes 4 outputs at a time,
+// so N must be a multiple of 4.
+int linear_split_k(int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (M <= kDecodeMaxM || N % 4 != 0 || K > sign_gemm_tc_max_k()) return 1;
+  return tc_split_k(M, N, K, num_sms);
+}
+
+ob_status ob_linear_ws(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,
+                       const float* b, void* Y, int y_dtype, void* workspace, size_t ws_bytes, int path,
+                       void* stream) {
   if (M < 0 || N < 0 || K < 0 || K % 32 != 0) return OB_ERR_SHAPE;
   if (!elems_ok(M, K) || !elems_ok(N, K) || !elems_ok(M, N)) return OB_ERR_SHAPE;
   if (y_dtype != OB_OUT_BF16 && y_dtype != OB_OUT_F32) return OB_ERR_UNSUPPORTED;
@@ -212,13 +226,38 @@ ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
   if (K > 0 && (!X || !W_packed || !b)) return OB_ERR_NULL;
   if (misaligned(Y) || misaligned(a) || (K > 0 && (misaligned(X) || misaligned(W_packed) || misaligned(b))))
     return OB_ERR_ALIGN;
+  if (workspace && misaligned(workspace)) return OB_ERR_ALIGN;
   LaunchCtx c;
   ob_status st = make_ctx(stream, &c);
   if (st != OB_OK) return st;
   if (K == 0) return zero_output(Y, M, N, y_dtype, c.stream);
   SignGemmArgs g{static_cast<const uint16_t*>(X), M, K, W_packed, N, b, a, Y, N, y_dtype};
   g.static_w = static_w;
+  // Few output tiles on the one-CTA tcgen05 GEMM (AUTO above the decode sizes where the CTA
+  // pair does not apply, OB_PATH_TC likewise, OB_PATH_TC1): split over K through the
+  // workspace when it holds the partial sums.  Measured on B200 at M = 256, K = N = 4096:
+  // 32 tiles on 32 SMs unsplit.
+  const bool one_cta = path == OB_PATH_TC1 ||
+                       ((path == OB_PATH_TC || (path == OB_PATH_AUTO && M > kDecodeMaxM)) &&
+                        !sign_gemm_tc2_supported(g));
+  if (one_cta && workspace) {
+    const int ks = linear_split_k(M, N, K, c.num_sms);
+    if (ks > 1 && ws_bytes >= (size_t)ks * (size_t)M * (size_t)N * 4)
+      return status_of(launch_sign_gemm_tc_splitk(g, ks, static_cast<float*>(workspace), c));
+  }
   return run_sign_gemm(g, path, c);
+}
+
+size_t ob_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0 || !elems_ok(M, K) || !elems_ok(N, K) || !elems_ok(M, N)) return 0;
+  if (M == 0 || N == 0 || K == 0) return 0;
+  const int ks = linear_split_k(M, N, K, sms_for_sizing());
+  return ks > 1 ? align256((size_t)ks * (size_t)M * (size_t)N * 4) : 0;
+}
+
+ob_status ob_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,
+                       const float* b, void* Y, int y_dtype, int path, void* stream) {
+  return ob_linear_ws(X, M, K, W_packed, N, a, b, Y, y_dtype, nullptr, 0, path, stream);
 }
 
 ob_status ob_linear(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,
@@ -281,14 +320,10 @@ size_t dbf_t_bytes(int64_t M, int64_t r) { return align256((size_t)M * (size_t)r
 // partial sums of a split product start after them.
 constexpr size_t kDbfBarrierBytes = 256;
 
-// K slices of DBF's first product (T = ... S_B^T, M x r) when it runs on the tcgen05 GEMM.
-int dbf_split_k(int64_t M, int64_t r, int num_sms) {
-  return M > kDecodeMaxM ? tc_split_k(M, r, num_sms) : 1;
-}
-
-int sms_for_sizing() {
-  DeviceInfo d;
-  return current_device(&d) == OB_OK && d.num_sms > 0 ? d.num_sms : 148;  // B200 when no device
+// K slices of DBF's first product (T = ... S_B^T, M x r, over K) when it runs on the tcgen05
+// GEMM; sizing does not know K, so it takes the most slices any K allows.
+int dbf_split_k(int64_t M, int64_t r, int num_sms, int64_t K = (int64_t)1 << 20) {
+  return M > kDecodeMaxM ? tc_split_k(M, r, K, num_sms) : 1;
 }
 
 size_t dbf_workspace_size(int64_t M, int64_t r) {
@@ -347,7 +382,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   // Few output tiles (small M x r): split the first product over K into fp32 partial
   // sums after T in the workspace, when the workspace holds them.
   const bool tc1 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > kDecodeMaxM && K <= sign_gemm_tc_max_k());
-  const int ks = tc1 ? dbf_split_k(M, r, c.num_sms) : 1;
+  const int ks = tc1 ? dbf_split_k(M, r, c.num_sms, K) : 1;
   const size_t part_off = t_bytes + kDbfBarrierBytes;
   if (ks > 1 && ws_bytes >= part_off + (size_t)ks * (size_t)M * (size_t)r * 4) {
     g1.l2_prefetch = 0;
@@ -367,7 +402,7 @@ ob_status dbf_linear_ex(const void* X, int64_t M, int64_t K, const uint32_t* SB_
   const bool tc2 = path == OB_PATH_TC || (path == OB_PATH_AUTO && M > kDecodeMaxM && r <= sign_gemm_tc_max_k());
   const bool pair2 = sign_gemm_tc2_supported(g2) && r < 4096;
   const int ks2 = (tc2 && !pair2 && M > kDecodeMaxM)
-                      ? tc_split_k(M, N, c.num_sms)
+                      ? tc_split_k(M, N, r, c.num_sms)
                       : 1;
   if (ks2 > 1 && ws_bytes >= part_off + (size_t)ks2 * (size_t)M * (size_t)N * 4)
     return status_of(launch_sign_gemm_tc_splitk(

@@ -479,10 +479,14 @@ int64_t sign_gemm_tc_max_k() { return kMaxK; }
 
 void* tensor_map_encode_tiled_fn() { return reinterpret_cast<void*>(get_encode_fn()); }
 
-int tc_split_k(int64_t M, int64_t R, int num_sms) {
+int tc_split_k(int64_t M, int64_t R, int64_t K, int num_sms) {
   const int64_t tiles = ((M + kTok - 1) / kTok) * ((R + kRows - 1) / kRows);
   if (tiles == 0 || tiles * 2 > num_sms) return 1;
-  return (int)std::min<int64_t>(8, num_sms / tiles);
+  // K slices are whole 4-stage groups, and at least 16 stages (1024 k) long: shorter
+  // slices cost more in the extra partial-sum pass than they gain (measured on B200).
+  const int64_t nkb = (K + kBK - 1) / kBK;
+  const int64_t ks = std::min<int64_t>(std::min<int64_t>(8, num_sms / tiles), std::min<int64_t>((nkb + 3) / 4, nkb / 16));
+  return ks > 1 ? (int)ks : 1;
 }
 
 namespace {
@@ -578,8 +582,7 @@ cudaError_t launch_sign_gemm_tc(const SignGemmArgs& g, const LaunchCtx& c) { ret
 
 cudaError_t launch_sign_gemm_tc_splitk(const SignGemmArgs& g, int ksplit, float* part, const LaunchCtx& c) {
   if (g.M == 0 || g.R == 0 || g.K == 0) return cudaSuccess;
-  // K slices are whole 4-stage groups, and at least 16 stages (1024 k) long: shorter
-  // slices cost more in the extra partial-sum pass than they gain (measured on B200).
+  // The same limits as tc_split_k: whole 4-stage groups of at least 16 stages.
   const int64_t nkb = (g.K + kBK - 1) / kBK;
   ksplit = (int)std::min<int64_t>(ksplit, std::min<int64_t>((nkb + 3) / 4, nkb / 16));
   if (ksplit <= 1 || g.R % 4 != 0 || g.ldy % 4 != 0) return launch_tc_impl(g, 1, nullptr, c);

@@ -54,7 +54,7 @@ cudaError_t launch_sign_gemm_tc2(const SignGemmArgs& g, const LaunchCtx& c);
 int64_t sign_gemm_tc_max_k();
 // K slices for the tcgen05 GEMM of an M x R output: more than one when the output has
 // fewer 128 x 256 tiles than half the SMs (at most 8).
-int tc_split_k(int64_t M, int64_t R, int num_sms);
+int tc_split_k(int64_t M, int64_t R, int64_t K, int num_sms);
 // The tcgen05 GEMM split over K: fp32 partial sums of each slice into part
 // (ksplit x M x R floats), then a reduction that applies oscale and writes Y.
 // Slices hold at least 1024 k; falls back to the unsplit kernel when K is too short for

@@ -90,10 +90,17 @@ def ob_svid_rank1(W: torch.Tensor, max_iters: int = 0, tol: float = 0.0, workspa
     return a, b, sigma, iters.value, st
 
 
+def ob_linear_workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib.lib().ob_linear_workspace_size(M, N, K))
+
+
 def ob_linear(X: torch.Tensor, W_packed: torch.Tensor, a: torch.Tensor, b: torch.Tensor,
               out_dtype: torch.dtype = torch.bfloat16, path: int = OB_PATH_AUTO, out: torch.Tensor | None = None,
-              stream=None) -> torch.Tensor:
-    """OneBit layer Y = [(X ⊙ b^T) W_sign^T] ⊙ a^T; X bf16 [M, K], W_packed int32 [N, K/32]."""
+              stream=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """OneBit layer Y = [(X ⊙ b^T) W_sign^T] ⊙ a^T; X bf16 [M, K], W_packed int32 [N, K/32].
+
+    workspace (uint8, optional): lets a few-tile tcgen05 problem split over K (ob_linear_ws).
+    """
     M, K = X.shape
     N = W_packed.shape[0]
     _need(X, "X", torch.bfloat16)
@@ -103,8 +110,13 @@ def ob_linear(X: torch.Tensor, W_packed: torch.Tensor, a: torch.Tensor, b: torch
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=X.device)
     _need(out, "out", out_dtype, (M, N))
-    st = _lib.lib().ob_linear_ex(_ptr(X), M, K, _ptr(W_packed), N, _ptr(a), _ptr(b), _ptr(out),
-                                 _out_code(out_dtype), int(path), _stream(stream))
+    if workspace is None:
+        st = _lib.lib().ob_linear_ex(_ptr(X), M, K, _ptr(W_packed), N, _ptr(a), _ptr(b), _ptr(out),
+                                     _out_code(out_dtype), int(path), _stream(stream))
+    else:
+        st = _lib.lib().ob_linear_ws(_ptr(X), M, K, _ptr(W_packed), N, _ptr(a), _ptr(b), _ptr(out),
+                                     _out_code(out_dtype), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     int(path), _stream(stream))
     _lib.check("ob_linear", st)
     return out
 

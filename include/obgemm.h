@@ -179,6 +179,28 @@ OB_API ob_status ob_linear(const void* X, int64_t M, int64_t K,
                     const float* a, const float* b,
                     void* Y, int y_dtype, void* stream);
 
+/* Bytes of device workspace ob_linear_ws can use for an M x K -> N layer: fp32 partial
+ * sums (slices x M x N x 4 bytes) when the layer would run on the one-CTA tcgen05 GEMM with
+ * fewer output tiles than half the SMs of the current device (e.g. M = 256, K = N = 4096),
+ * N % 4 == 0 and K holds at least two slices of 1024; 0 when no split applies.  An upper
+ * bound: the output dtype is not known here, and a bf16 layer that the CTA pair takes
+ * (M >= 512, N >= 256, K <= 16384) runs unsplit. */
+OB_API size_t ob_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * ob_linear_ex with a caller workspace.  Where the layer runs on the one-CTA tcgen05 GEMM
+ * (OB_PATH_AUTO above 16 tokens when the CTA pair does not apply, OB_PATH_TC likewise,
+ * OB_PATH_TC1) with few output tiles, K is split into slices whose fp32 partial sums go to
+ * the workspace; a second kernel sums them, applies a and stores Y.  A workspace smaller than
+ * ob_linear_workspace_size (or NULL with ws_bytes 0) runs unsplit.
+ *   workspace  device, 16-byte aligned, or NULL; not shared with a concurrent call.
+ * Otherwise as ob_linear_ex.
+ */
+OB_API ob_status ob_linear_ws(const void* X, int64_t M, int64_t K,
+                       const uint32_t* W_packed, int64_t N,
+                       const float* a, const float* b,
+                       void* Y, int y_dtype, void* workspace, size_t ws_bytes, int path, void* stream);
+
 /* ob_linear with an explicit kernel choice (ob_path). */
 OB_API ob_status ob_linear_ex(const void* X, int64_t M, int64_t K,
                        const uint32_t* W_packed, int64_t N,

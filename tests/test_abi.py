@@ -52,6 +52,23 @@ def test_status_strings_and_version(lib):
     assert lib.ob_version() >= 10000
 
 
+def test_linear_workspace_size_and_checks(lib):
+    # fp32 partial sums of the K slices for few-tile tcgen05 problems; 0 where no split applies
+    assert lib.ob_linear_workspace_size(256, 4096, 4096) == 4 * 256 * 4096 * 4   # 32 tiles: 4 slices
+    assert lib.ob_linear_workspace_size(16, 4096, 4096) == 0     # decode sizes
+    assert lib.ob_linear_workspace_size(256, 4098, 4096) == 0    # N % 4 != 0
+    assert lib.ob_linear_workspace_size(2048, 11008, 4096) == 0  # enough tiles
+    assert lib.ob_linear_workspace_size(256, 4096, 40960) == 0   # K past the tcgen05 limit
+    assert lib.ob_linear_workspace_size(-1, 4096, 4096) == 0
+    assert lib.ob_linear_workspace_size(1 << 40, 1 << 40, 32) == 0
+    OK, NULL, SHAPE, ALIGN, UNSUP = 0, 1, 2, 3, 9
+    p, bad = ctypes.c_void_p(4096), ctypes.c_void_p(4100)
+    assert lib.ob_linear_ws(p, 256, 64, p, 4, p, p, p, 0, bad, 1 << 20, 0, None) == ALIGN
+    assert lib.ob_linear_ws(p, 256, 48, p, 4, p, p, p, 0, p, 1 << 20, 0, None) == SHAPE
+    assert lib.ob_linear_ws(p, 256, 64, p, 4, p, p, p, 0, p, 1 << 20, 6, None) == UNSUP
+    assert lib.ob_linear_ws(None, 0, 64, None, 4, None, None, None, 0, None, 0, 0, None) == OK
+
+
 def test_workspace_sizes(lib):
     assert lib.dbf_workspace_size(512, 2048) >= 512 * 2048 * 2
     assert lib.dbf_workspace_size(0, 32) == 0

@@ -219,6 +219,35 @@ def test_sweep_with_outliers(ops, shape_idx, M):
     assert_gemm_close(Y, _ref(x, W, a, b), what=f"sweep {K}->{N} M={M}")
 
 
+@pytest.mark.parametrize("M,N,K,path", [(256, 4096, 4096, 0), (64, 1024, 2048, 0), (300, 512, 11008, 0),
+                                        (128, 2048, 8192, 0), (17, 1000, 160, 0), (256, 4096, 4096, 7),
+                                        (600, 512, 2048, 0), (256, 132, 512, 0)])
+def test_linear_ws_split_over_k(ops, M, N, K, path):
+    # ob_linear_ws: few output tiles on the one-CTA tcgen05 GEMM split over K through the
+    # workspace (fp32 partial sums); every element against the oracle; a workspace one byte
+    # short, and none, run unsplit with the same result.
+    from helpers import Guarded
+    W = synth.weights(M + N + K, N, K)
+    a, b, _ = oracle.svid_rank1(W)
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    xb, x = synth.activations(M + K, M, K)
+    P = ops.ob_pack_signs(_cuda(W))
+    X, A, B = _x_bf16(xb), _cuda(a), _cuda(b)
+    ref = _ref(x, W, a, b)
+    need = ops.ob_linear_workspace_size(M, N, K)
+    for ws_bytes in sorted({need, max(need - 1, 0), 0}):
+        ws = Guarded((max(ws_bytes, 1),), torch.uint8) if ws_bytes else None
+        out = Guarded((M, N), torch.bfloat16)
+        ops.ob_linear(X, P, A, B, out=out.t, path=path,
+                      workspace=None if ws is None else ws.t[:ws_bytes] if ws_bytes else None)
+        torch.cuda.synchronize()
+        assert ops.ob_last_device_error() == 0
+        out.check("ob_linear_ws output")
+        if ws is not None:
+            ws.check("ob_linear_ws workspace")
+        assert_gemm_close(out.t, ref, what=f"ob_linear_ws {M}x{N}x{K} path {path} ws {ws_bytes}")
+
+
 def test_cuda_graph_replay_matches(ops):
     W, a, b, _ = oracle_svid(1, 4096, 4096)
     xb, x = synth.activations(1, 4, 4096)
