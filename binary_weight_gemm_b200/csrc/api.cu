@@ -121,6 +121,19 @@ constexpr int64_t kFactorizeMaxDim = (int64_t)1 << 22;
 constexpr int64_t kMaxElems = (int64_t)1 << 48;
 bool elems_ok(int64_t rows, int64_t cols) { return rows == 0 || cols <= kMaxElems / rows; }
 
+int sms_for_sizing() {
+  DeviceInfo d;
+  return current_device(&d) == OB_OK && d.num_sms > 0 ? d.num_sms : 148;  // B200 when no device
+}
+
+// K slices for a problem that runs on the one-CTA tcgen05 GEMM with few output tiles (1: no
+// split).  The slices' partial sums are summed by a kernel that writes 4 outputs at a time,
+// so N must be a multiple of 4.
+int linear_split_k(int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (M <= kDecodeMaxM || N % 4 != 0 || K > sign_gemm_tc_max_k()) return 1;
+  return tc_split_k(M, N, K, num_sms);
+}
+
 }  // namespace
 }  // namespace ob
 
@@ -196,19 +209,6 @@ ob_status ob_svid_rank1(const float* W, int64_t N, int64_t K, float* a, float* b
   ob_status st = make_ctx(stream, &c);
   if (st != OB_OK) return st;
   return run_svid(W, N, K, a, b, sigma1, max_iters, tol, iters_out, workspace, c);
-}
-
-int sms_for_sizing() {
-  DeviceInfo d;
-  return current_device(&d) == OB_OK && d.num_sms > 0 ? d.num_sms : 148;  // B200 when no device
-}
-
-// K slices for a problem that runs on the one-CTA tcgen05 GEMM with few output tiles (1: no
-// split).  The slices' partial sums are summed by a kernel that writes 4 outputs at a time,
-// so N must be a multiple of 4.
-int linear_split_k(int64_t M, int64_t N, int64_t K, int num_sms) {
-  if (M <= kDecodeMaxM || N % 4 != 0 || K > sign_gemm_tc_max_k()) return 1;
-  return tc_split_k(M, N, K, num_sms);
 }
 
 ob_status ob_linear_ws(const void* X, int64_t M, int64_t K, const uint32_t* W_packed, int64_t N, const float* a,

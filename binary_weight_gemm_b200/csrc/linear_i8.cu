@@ -9,13 +9,12 @@
 //
 // A CTA owns RT = 2 row tiles (32 rows) and all of K, taken in chunks of super-blocks
 // (512 k) that fit shared memory.  Per chunk: every warp requests the packed words of its
-// items (row tile warp % 2, super-blocks warp / 2, + 4, ...); the CTA stages the chunk's
-// activation limbs (per (token, super-block) pair: largest |x'| first, then, once the
-// chunk's scale is known, the quantised limbs); the warps multiply, keeping exact int32
-// sums per bit position, and fold them into fp32 at the end of the chunk.  The warps of
-// a row tile are summed in shared memory, T (the sum of x') is added, then the output
-// scale and the store.
-//
+// items (row tile warp % 2, super-blocks warp / 2, + 4, ...); each warp stages (token,
+// super-block) pairs on its own (largest |x'|, the pair's scale, the quantised limbs); the
+// warps multiply, keeping exact int32 sums per (tile, super-block), and fold them into fp32
+// with the super-block's factors.  The warps of a row tile are summed in shared memory, T
+// (the sum of x') is added, then the output scale and the store.
+
 // Programmatic dependent launch: before griddepcontrol.wait a CTA only prefetches its
 // sign rows into L2 (every input may be an output of the previous grid); the next grid
 // is released after the wait.
