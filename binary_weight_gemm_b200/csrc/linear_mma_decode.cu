@@ -23,9 +23,7 @@
 //  * B (16 x 8) = the same 16 k x 8 tokens of x (bf16, exact), copied by each
 //    warp into shared memory already in fragment order and permuted the same
 //    way (one byte permutation per register), so the MMA contracts matching k.
-//    A CTA takes up to 8 tokens (one n8 tile); 9 to 16 tokens run on a grid of two CTA
-//    rows, each with half of them (the 16-token block, two n8 tiles, serves the layer
-//    stack).
+//    M <= 8 uses one n8 tile, M <= 16 two.
 //  * Each tile keeps 2-4 independent accumulator sets (word w goes to set
 //    w mod sets) so consecutive MMAs do not wait on each other.
 //  * A CTA owns 32 weight rows (two m16 tiles); its 8 warps take 512-k chunks of
@@ -52,13 +50,11 @@ namespace {
 using namespace mmad;
 
 // TOK: tokens per pass the kernel is built for (1, 8 or 16).  One CTA per 32-row block.
-// grid.y > 1: CTA (x, y) takes tokens m0 + TOK y .. m0 + TOK y + TOK - 1 of the same rows.
 template <int TOK, bool kVec>
 __global__ void __launch_bounds__(kThreads, TOK > 8 ? 1 : 2) sign_gemm_mma_decode_kernel(SignGemmArgs g, int64_t m0) {
   extern __shared__ __align__(16) uint8_t dsm[];
   __shared__ BlockShared<TOK> shb;
   const int64_t n0 = (int64_t)blockIdx.x * kRowsPerCta;
-  m0 += (int64_t)blockIdx.y * TOK;
   // Before the previous grid has finished, only pull this CTA's sign rows (one
   // contiguous block) into L2; the reads themselves come after pdl_wait.  With static
   // weights (the previous grid did not write them) each warp's first chunk of sign
@@ -76,9 +72,9 @@ __global__ void __launch_bounds__(kThreads, TOK > 8 ? 1 : 2) sign_gemm_mma_decod
 }
 
 template <int TOK, bool kVec>
-cudaError_t launch_tok(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c, unsigned ny = 1) {
+cudaError_t launch_tok(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((g.R + kRowsPerCta - 1) / kRowsPerCta), ny, 1);
+  cfg.gridDim = dim3((unsigned)((g.R + kRowsPerCta - 1) / kRowsPerCta), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   const size_t smem = dyn_smem_bytes<TOK>();
   cfg.dynamicSmemBytes = smem;
@@ -98,14 +94,11 @@ cudaError_t launch_tok(const SignGemmArgs& g, int64_t m0, const LaunchCtx& c, un
   return cudaLaunchKernelEx(&cfg, kern, g, m0);
 }
 
-// 9..16 tokens: the 8-token build on a two-row grid (each CTA one half of the tokens), which
-// keeps two CTAs per SM; the 16-token build (one CTA per SM for its shared memory) measured
-// slower per call at M = 16, K = N = 4096.
 template <bool kVec>
 cudaError_t launch_vec(const SignGemmArgs& g, int64_t m0, int64_t mt, const LaunchCtx& c) {
   if (mt == 1) return launch_tok<1, kVec>(g, m0, c);
   if (mt <= 8) return launch_tok<8, kVec>(g, m0, c);
-  return launch_tok<8, kVec>(g, m0, c, 2);
+  return launch_tok<16, kVec>(g, m0, c);
 }
 
 }  // namespace
