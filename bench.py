@@ -721,6 +721,32 @@ def run_stack(args, world, rank, local):
 
     specs = {m: spec(m) for m in ms_list}
     ws = torch.zeros(ops.ob_stack_workspace_size(), dtype=torch.uint8, device=dev)
+
+    # The dataflow form (int8, M <= 2): every layer of every block writes its own buffer, so
+    # the list qualifies; consumers poll their producers' tagged outputs, no grid barriers.
+    df_ms = [m for m in ms_list if m <= 2]
+
+    def spec_df(m):
+        x0, _ = acts[m]
+        out, x = [], x0
+        for bi, L in enumerate(layers):
+            bb = {name: torch.empty((m, N), dtype=torch.bfloat16, device=dev) for name, (K, N) in STACK_SHAPES.items()}
+            for name in ("q", "k", "v"):
+                P, a, b = L[name]
+                out.append((x, P, a, b, bb[name], bi > 0 and name == "q"))
+            P, a, b = L["o"]
+            out.append((bb["q"], P, a, b, bb["o"], True))
+            for name in ("gate", "up"):
+                P, a, b = L[name]
+                out.append((bb["o"], P, a, b, bb[name], name == "gate"))
+            P, a, b = L["down"]
+            out.append((bb["gate"], P, a, b, bb["down"], True))
+            x = bb["down"]
+        return out
+
+    dspecs = {m: spec_df(m) for m in df_ms}
+    dws = {m: torch.zeros(ops.ob_linear_stack_workspace_size(dspecs[m], m), dtype=torch.uint8, device=dev)
+           for m in df_ms}
     graphs, pgraphs = {}, {}
     with torch.cuda.stream(stream):
         for m in ms_list:
@@ -734,6 +760,13 @@ def run_stack(args, world, rank, local):
             pgraphs[m] = torch.cuda.CUDAGraph()
             with torch.cuda.graph(pgraphs[m], stream=stream):
                 ops.ob_linear_stack(specs[m], m, workspace=ws, stream=stream)
+        dgraphs = {}
+        for m in df_ms:
+            ops.ob_linear_stack(dspecs[m], m, workspace=dws[m], stream=stream)
+            stream.synchronize()
+            dgraphs[m] = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(dgraphs[m], stream=stream):
+                ops.ob_linear_stack(dspecs[m], m, workspace=dws[m], stream=stream)
         # The bf16 warp-MMA stack form forced at one token, beside the int8 form AUTO takes.
         mgraphs = {}
         ops.ob_linear_stack(specs[1], 1, workspace=ws, stream=stream, path=ops.OB_PATH_MMA_DECODE)
@@ -749,7 +782,8 @@ def run_stack(args, world, rank, local):
 
     ms_max, ms, clocks = _timed(step, args, world, stream, local)
     per_m = {}
-    for mode, gs in (("persistent", pgraphs), ("per_call", graphs), ("persistent_bf16mma", mgraphs)):
+    for mode, gs in (("persistent", pgraphs), ("per_call", graphs), ("persistent_bf16mma", mgraphs),
+                     ("persistent_dataflow", dgraphs)):
         for m in gs:
             reps = max(3, args.steps // 2)
             with torch.cuda.stream(stream):
@@ -783,7 +817,9 @@ def run_stack(args, world, rank, local):
                                 "grid barriers between dependent layers; AUTO: int8 form at M=1 and 2, bf16 "
                                 "warp-MMA form at M=16; persistent_bf16mma_M1 forces the bf16 form); per_call_* "
                                 "times one ob_linear per layer (AUTO | OB_FLAG_STATIC_WEIGHTS) in a graph with "
-                                "programmatic dependent launch",
+                                "programmatic dependent launch; persistent_dataflow_* gives every layer its own "
+                                "output buffer and the workspace of ob_linear_stack_workspace_size (tagged outputs "
+                                "polled by their consumers instead of grid barriers)",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "per_m": per_m,
             "gpu_launches": args.steps * len(ms_list), "clocks": clocks, "cpu_baseline": None,

@@ -47,6 +47,7 @@ SIGNATURES = {
     "ob_linear_ws": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _P, _SZ, _I, _P]),
     "ob_linear_ln": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _P, _I, _F, _I, _P]),
     "ob_stack_workspace_size": (_SZ, []),
+    "ob_linear_stack_workspace_size": (_SZ, [ctypes.POINTER(ObLayer), _I, _I64]),
     "ob_linear_stack": (_I, [ctypes.POINTER(ObLayer), _I, _I64, _P, _SZ, _P]),
     "ob_linear_stack_ex": (_I, [ctypes.POINTER(ObLayer), _I, _I64, _P, _SZ, _I, _P]),
     "dbf_workspace_size": (_SZ, [_I64, _I64]),

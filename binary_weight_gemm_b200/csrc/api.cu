@@ -279,6 +279,18 @@ ob_status ob_linear_ln(const void* X, int64_t M, int64_t K, const uint32_t* W_pa
 
 size_t ob_stack_workspace_size(void) { return 256; }
 
+size_t ob_linear_stack_workspace_size(const ob_layer* layers, int n_layers, int64_t M) {
+  const size_t base = ob_stack_workspace_size();
+  if (!layers || n_layers <= 0 || M < 1 || M > kStackI8MaxM) return base;
+  std::vector<StackLayerHost> host((size_t)n_layers);
+  for (int i = 0; i < n_layers; ++i) {
+    const ob_layer& L = layers[i];
+    if (L.K < 32 || L.N < 1 || L.N > ((int64_t)1 << 35) || !elems_ok(L.N, L.K)) return base;
+    host[i] = StackLayerHost{L.X, L.W_packed, L.b, L.a, L.Y, L.K, L.N, L.y_dtype, L.after_previous ? 1 : 0};
+  }
+  return base + align256(stack_tag_words(host.data(), n_layers, M) * sizeof(uint32_t));
+}
+
 ob_status ob_linear_stack_ex(const ob_layer* layers, int n_layers, int64_t M, void* workspace, size_t ws_bytes,
                              int path, void* stream) {
   if (n_layers < 0 || M < 0 || M > kDecodeMaxM) return OB_ERR_SHAPE;
@@ -305,7 +317,16 @@ ob_status ob_linear_stack_ex(const ob_layer* layers, int n_layers, int64_t M, vo
   ob_status st = make_ctx(stream, &c);
   if (st != OB_OK) return st;
   if (path == OB_PATH_AUTO) path = M <= kStackI8MaxM ? OB_PATH_I8 : OB_PATH_MMA_DECODE;
-  return status_of(launch_sign_stack(host.data(), n_layers, M, static_cast<unsigned*>(workspace), c, path));
+  // A workspace beyond the barrier words holds the tagged outputs of the dataflow form.
+  const size_t base = ob_stack_workspace_size();
+  uint32_t* tags = nullptr;
+  size_t tag_words = 0;
+  if (path == OB_PATH_I8 && ws_bytes > base) {
+    tags = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + base);
+    tag_words = (ws_bytes - base) / sizeof(uint32_t);
+  }
+  return status_of(
+      launch_sign_stack(host.data(), n_layers, M, static_cast<unsigned*>(workspace), c, path, tags, tag_words));
 }
 
 ob_status ob_linear_stack(const ob_layer* layers, int n_layers, int64_t M, void* workspace, size_t ws_bytes,

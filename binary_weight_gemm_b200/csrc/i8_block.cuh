@@ -111,6 +111,30 @@ __device__ __forceinline__ StageRaw stage_load(const SignGemmArgs& g, int64_t m_
   return r;
 }
 
+// Stage a pair from tagged words instead of X: word k of token m is kTagMark | bf16 bits at
+// tags[m * K + k], written by an earlier layer of the same launch.  Loads the lane's words
+// (relaxed, from L2) and its input scales into r; returns whether all of the lane's words
+// carry the mark (words past K or of a token not present count as ready).
+__device__ __forceinline__ bool stage_load_tagged(const SignGemmArgs& g, const uint32_t* tags, int64_t m_glob,
+                                                  bool live, int64_t kbase, int lane, StageRaw& r) {
+  const int q = lane >> 1, jh = (lane & 1) * 4;
+  const int64_t K = g.K;
+  bool ready = true;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t k0 = kbase + 32 * q + 8 * i + jh;
+    r.sc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    r.x[i] = make_uint2(0u, 0u);
+    if (live && k0 < K) {
+      r.sc[i] = g.iscale ? __ldg(reinterpret_cast<const float4*>(g.iscale + k0)) : make_float4(1.f, 1.f, 1.f, 1.f);
+      const uint4 w = ld_volatile_v4(tags + m_glob * K + k0);
+      ready &= ((w.x & w.y & w.z & w.w) >> 16) == (kTagMark >> 16) && ((w.x | w.y | w.z | w.w) >> 16) == (kTagMark >> 16);
+      r.x[i] = make_uint2(__byte_perm(w.x, w.y, 0x5410), __byte_perm(w.z, w.w, 0x5410));
+    }
+  }
+  return ready;
+}
+
 // x' of the lane's 16 values: v[i][jj] at k = kbase + 32 q + 8 i + jh + jj.
 __device__ __forceinline__ void stage_values(const StageRaw& raw, float (&v)[4][4]) {
 #pragma unroll

@@ -21,6 +21,7 @@
 //    its wait is bounded: a CTA that gives up records a timeout in the error
 //    word and sets an abort word that makes every other CTA leave at its next barrier.
 #include <algorithm>
+#include <vector>
 #include <cstring>
 
 #include "mma_decode_block.cuh"
@@ -119,13 +120,64 @@ cudaError_t launch_stack_tok(const StackParams& prm, const LaunchCtx& c) {
 
 int stack_max_layers_per_launch() { return kStackMaxLayers; }
 
+namespace {
+
+// The dataflow plan of one launch's layers [0, n): producer of each layer's input (-1: an
+// input from outside the launch) and tag offsets (words; -1: no consumer).  Returns the tag
+// words needed, or -1 when the launch does not qualify (an output overlaps another output,
+// or an input that is not exactly an earlier layer's bf16 output).
+int64_t dataflow_plan(const StackLayerHost* L, int n, int64_t M, std::vector<int>& prod, std::vector<int64_t>& off) {
+  prod.assign((size_t)n, -1);
+  off.assign((size_t)n, -1);
+  auto ybytes = [&](int i) { return (uintptr_t)(M * L[i].N * (L[i].y_dtype == OB_OUT_F32 ? 4 : 2)); };
+  auto xbytes = [&](int i) { return (uintptr_t)(M * L[i].K * 2); };
+  auto overlap = [](uintptr_t a, uintptr_t an, uintptr_t b, uintptr_t bn) { return a < b + bn && b < a + an; };
+  for (int j = 0; j < n; ++j) {
+    const uintptr_t xj = reinterpret_cast<uintptr_t>(L[j].X), yj = reinterpret_cast<uintptr_t>(L[j].Y);
+    for (int i = j - 1; i >= 0 && prod[j] < 0; --i)
+      if (reinterpret_cast<uintptr_t>(L[i].Y) == xj && L[i].y_dtype == OB_OUT_BF16 && ybytes(i) == xbytes(j))
+        prod[j] = i;
+    for (int i = 0; i < n; ++i) {
+      const uintptr_t yi = reinterpret_cast<uintptr_t>(L[i].Y);
+      if (i != j && overlap(yi, ybytes(i), yj, ybytes(j))) return -1;          // two layers write one buffer
+      if (overlap(yi, ybytes(i), xj, xbytes(j)) && i != prod[j]) return -1;    // not a producer's output
+    }
+  }
+  // Each tagged output starts on a 256-byte boundary: consumers read it 16 bytes at a time.
+  int64_t words = 0;
+  for (int j = 0; j < n; ++j)
+    if (prod[j] >= 0 && off[(size_t)prod[j]] < 0) {
+      off[(size_t)prod[j]] = words;
+      words += (M * L[prod[j]].N + 63) & ~(int64_t)63;
+    }
+  return words;
+}
+
+}  // namespace
+
+size_t stack_tag_words(const StackLayerHost* layers, int n, int64_t M) {
+  if (M < 1 || M > 2) return 0;  // the int8 form
+  size_t most = 0;
+  std::vector<int> prod;
+  std::vector<int64_t> off;
+  for (int base = 0; base < n; base += kStackMaxLayers) {
+    const int cnt = std::min(kStackMaxLayers, n - base);
+    const int64_t w = dataflow_plan(layers + base, cnt, M, prod, off);
+    if (w < 0) return 0;  // one launch of the list would need barriers: no dataflow for the list
+    most = std::max(most, (size_t)w);
+  }
+  return most;
+}
+
 cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c,
-                              int path) {
+                              int path, uint32_t* tags, size_t tag_words) {
   if (n == 0 || M == 0) return cudaSuccess;
   static_assert(sizeof(StackParams) <= 32000, "kernel parameters");
   StackParams* prm = new StackParams;
   std::memset(prm, 0, sizeof(StackParams));
   cudaError_t e = cudaSuccess;
+  std::vector<int> prod;
+  std::vector<int64_t> off;
   for (int base = 0; base < n && e == cudaSuccess; base += kStackMaxLayers) {
     const int cnt = std::min(kStackMaxLayers, n - base);
     prm->n = cnt;
@@ -137,11 +189,23 @@ cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, un
       const int nb = (int)((h.N + kRowsPerCta - 1) / kRowsPerCta);
       const int vec = ((h.K / 32) % 4 == 0) && ((reinterpret_cast<uintptr_t>(h.S) & 15) == 0);
       prm->L[i] = StackLayer{static_cast<const uint16_t*>(h.X), h.S, h.iscale, h.oscale, h.Y, h.K, h.N, h.y_dtype,
-                             i == 0 ? 0 : h.barrier, nb, vec};
+                             i == 0 ? 0 : h.barrier, nb, vec, nullptr, nullptr};
     }
+    const bool i8 = path == OB_PATH_I8 && stack_i8_supported(*prm);
+    // Dataflow: the int8 form, a tag area, and a launch that qualifies.
+    int64_t words = -1;
+    if (i8 && tags) words = dataflow_plan(layers + base, cnt, M, prod, off);
+    prm->dataflow = (words >= 0 && (size_t)words <= tag_words) ? 1 : 0;
+    if (prm->dataflow)
+      for (int i = 0; i < cnt; ++i) {
+        if (off[(size_t)i] >= 0) prm->L[i].tag_out = tags + off[(size_t)i];
+        if (prod[(size_t)i] >= 0) prm->L[i].tag_in = tags + off[(size_t)prod[(size_t)i]];
+      }
     e = cudaMemsetAsync(bar, 0, 2 * sizeof(unsigned), c.stream);
+    if (e == cudaSuccess && prm->dataflow && words > 0)
+      e = cudaMemsetAsync(tags, 0, (size_t)words * sizeof(uint32_t), c.stream);  // no word is ready yet
     if (e != cudaSuccess) break;
-    if (path == OB_PATH_I8 && stack_i8_supported(*prm))
+    if (i8)
       e = launch_stack_i8(*prm, c);
     else
       e = M == 1 ? launch_stack_tok<1>(*prm, c) : (M <= 8 ? launch_stack_tok<8>(*prm, c) : launch_stack_tok<16>(*prm, c));

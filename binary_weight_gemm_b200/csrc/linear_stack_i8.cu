@@ -166,11 +166,11 @@ __device__ void fetch_seg(const StackLayer& L, const Seg& s, uint32_t* wbuf, uin
 }
 
 // The last warp copies layer li's descriptor from the parameter block into shared memory
-// (18 words, one per lane).  The caller makes the copy visible (a CTA barrier, or
+// (22 words, one per lane).  The caller makes the copy visible (a CTA barrier, or
 // __syncwarp for the same warp) before it is read.
-static_assert(sizeof(StackLayer) == 72, "a layer descriptor is 18 words");
+static_assert(sizeof(StackLayer) == 88, "a layer descriptor is 22 words");
 __device__ __forceinline__ void load_desc(const StackParams& p, int li, StackLayer* dst, int lane) {
-  if (lane < 18) reinterpret_cast<uint32_t*>(dst)[lane] = reinterpret_cast<const uint32_t*>(&p.L[li])[lane];
+  if (lane < 22) reinterpret_cast<uint32_t*>(dst)[lane] = reinterpret_cast<const uint32_t*>(&p.L[li])[lane];
 }
 
 // Packed words of row `row` (relative to the segment) for a super-block: words w0 .. w0+3.
@@ -310,10 +310,44 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
           // Staging: the pairs (token, super-block) p = warp, warp + 8, warp + 16, each with
           // its own scale; then warp 7 sums T while the others start multiplying.
           StageRaw raw[kMaxPairs];
+          if (L.tag_in) {
+            // Dataflow: the input is an earlier layer's tagged output; poll the pairs' words
+            // until every one carries the mark (the area was zeroed before the launch).
+            bool in_ok = true;
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t it = 0;; ++it) {
+              bool ready = true;
 #pragma unroll
-          for (int k = 0; k < kMaxPairs; ++k) {
-            const int pp = warp + k * kWarps;
-            if (pp < TOK * chn) raw[k] = stage_load<true>(g, pp % TOK, pp % TOK < mt, (sb0 + pp / TOK) * kSbK, lane);
+              for (int k = 0; k < kMaxPairs; ++k) {
+                const int pp = warp + k * kWarps;
+                if (pp < TOK * chn)
+                  ready &= stage_load_tagged(g, L.tag_in, pp % TOK, pp % TOK < mt, (sb0 + pp / TOK) * kSbK, lane,
+                                             raw[k]);
+              }
+              if (__all_sync(0xffffffffu, ready)) break;
+              if ((it & 15u) == 15u) {
+                if (ld_acquire_gpu(p.bar + 1) != 0u) {
+                  in_ok = false;
+                  break;
+                }
+                if (globaltimer_ns() - t0 > OB_WAIT_LIMIT_NS || it > (1u << 24)) {
+                  if (lane == 0) {
+                    record_error(p.err, OB_DEVERR_TIMEOUT);
+                    atomicExch(p.bar + 1, 1u);
+                  }
+                  in_ok = false;
+                  break;
+                }
+              }
+              __nanosleep(32);
+            }
+            if (!in_ok && lane == 0) s_abort = 1;
+          } else {
+#pragma unroll
+            for (int k = 0; k < kMaxPairs; ++k) {
+              const int pp = warp + k * kWarps;
+              if (pp < TOK * chn) raw[k] = stage_load<true>(g, pp % TOK, pp % TOK < mt, (sb0 + pp / TOK) * kSbK, lane);
+            }
           }
 #pragma unroll
           for (int k = 0; k < kMaxPairs; ++k) {
@@ -433,15 +467,19 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
         }
         v *= osc[j];
         const int64_t off = (int64_t)m * L.N + n;
-        if (L.y_dtype == OB_OUT_F32)
+        if (L.y_dtype == OB_OUT_F32) {
           static_cast<float*>(L.Y)[off] = v;
-        else
-          static_cast<__nv_bfloat16*>(L.Y)[off] = __float2bfloat16_rn(v);
+        } else {
+          const __nv_bfloat16 yb = __float2bfloat16_rn(v);
+          static_cast<__nv_bfloat16*>(L.Y)[off] = yb;
+          if (L.tag_out) st_volatile_u32(L.tag_out + off, kTagMark | (uint32_t)__bfloat16_as_ushort(yb));
+        }
       }
       cur ^= 1;
     }
     staged = -1;  // the next group's inputs are new
-    if (gi + 1 < ng) {
+    // Dataflow launches have no grid barrier: a consumer polls its producer's tagged output.
+    if (gi + 1 < ng && !p.dataflow) {
       ++barriers;
       // While thread 0 waits, the copy thread requests the scale vectors of the group after
       // the next into L2 (the next group's were requested with its weights, which is late for

@@ -16,6 +16,10 @@ struct LaunchCtx {
   bool l2_prefetch;  // with pdl: prefetch the weights into L2 before waiting on the previous grid
 };
 
+// High half of a tagged output word (kTagMark | bf16 bits) of the dataflow form of the
+// int8 layer stack; its tag area is zeroed before every launch, so a zero word is not ready.
+constexpr uint32_t kTagMark = 0xA5A50000u;
+
 // One sign-product layer  Y[m, n] = oscale[n] * sum_k (x[m, k] * iscale[k]) * s[n, k],
 // with s the packed sign matrix (R x K, R = output features).  X is bf16 M x K
 // (row stride K); iscale may be null (no input scale).  Y is M x R with row
@@ -91,9 +95,16 @@ struct StackLayerHost {
 // Runs the list (M <= 16) as cooperative launches of at most stack_max_layers_per_launch()
 // layers; bar: 8 bytes of device memory (zeroed by the launcher).  path: OB_PATH_I8 (M <= 2)
 // for the int8 form, OB_PATH_MMA_DECODE for the bf16 form.
+// tags / tag_words: device area for tagged outputs (dataflow launches of the int8 form, where
+// stack_tag_words() says the list allows them), or null / 0 for grid barriers only.
 cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, unsigned* bar, const LaunchCtx& c,
-                              int path);
+                              int path, uint32_t* tags = nullptr, size_t tag_words = 0);
 int stack_max_layers_per_launch();
+// 32-bit words of tagged outputs a dataflow launch of the list needs (the largest over its
+// launches), or 0 when no launch of it qualifies: every layer writes its own buffer, and
+// every input is either outside all outputs of its launch or exactly the bf16 output of an
+// earlier layer of it.
+size_t stack_tag_words(const StackLayerHost* layers, int n, int64_t M);
 
 // Z = LayerNorm(Y) per row of the M x N matrix Y (row stride ld elements), in place.
 cudaError_t launch_layernorm_rows(void* Y, int64_t M, int64_t N, int64_t ld, int y_dtype, float eps,

@@ -26,15 +26,21 @@ struct StackLayer {
   int32_t barrier;  // wait for every earlier layer of the list before this one
   int32_t nb;       // 32-row blocks: ceil(N / 32)
   int32_t vec;      // the sign rows allow 16-byte copies
+  // Tagged outputs (int8 form, dataflow launches only): each output also written as a
+  // 32-bit word kTagMark | bf16 bits into tag_out, which a consuming layer of the same
+  // launch polls (tag_in) instead of waiting at a grid barrier.  Null otherwise.
+  uint32_t* tag_out;
+  const uint32_t* tag_in;
 };
 
-constexpr int kStackMaxLayers = 384;  // 384 x 72 B of kernel parameters
+constexpr int kStackMaxLayers = 320;  // 320 x 88 B of kernel parameters
 
 struct StackParams {
   int n;
   int64_t M;
   unsigned* bar;  // [0] arrivals, [1] abort
   unsigned* err;
+  int dataflow;   // tagged outputs replace the grid barriers (see StackLayer::tag_out)
   StackLayer L[kStackMaxLayers];
 };
 

@@ -144,15 +144,7 @@ def ob_stack_workspace_size() -> int:
     return int(_lib.lib().ob_stack_workspace_size())
 
 
-def ob_linear_stack(layers, M: int, workspace: torch.Tensor | None = None, stream=None,
-                    path: int = OB_PATH_AUTO) -> None:
-    """Run a list of OneBit layers (M <= 16 tokens) in one persistent launch.
-
-    layers: sequence of (X, W_packed, a, b, Y, after_previous); X bf16 [M, K], W_packed int32
-    [N, K/32], a fp32 [N], b fp32 [K] or None, Y bf16/fp32 [M, N] (written), after_previous:
-    True if X is an output of an earlier layer of the list.  path: OB_PATH_AUTO,
-    OB_PATH_MMA_DECODE or OB_PATH_I8 (M <= 2).
-    """
+def _stack_array(layers, M: int):
     arr = (_lib.ObLayer * max(1, len(layers)))()
     dev = None
     for i, (X, P, a, b, Y, after) in enumerate(layers):
@@ -167,6 +159,27 @@ def ob_linear_stack(layers, M: int, workspace: torch.Tensor | None = None, strea
         arr[i] = _lib.ObLayer(_ptr(X), _ptr(P), _ptr(a), _ptr(b), _ptr(Y), K, N, _out_code(Y.dtype),
                               1 if after else 0)
         dev = X.device
+    return arr, dev
+
+
+def ob_linear_stack_workspace_size(layers, M: int) -> int:
+    """Workspace bytes with which ob_linear_stack runs this list in its dataflow form (tagged
+    outputs instead of grid barriers; int8 form, M <= 2), or ob_stack_workspace_size()."""
+    arr, _ = _stack_array(layers, M)
+    return int(_lib.lib().ob_linear_stack_workspace_size(arr, len(layers), M))
+
+
+def ob_linear_stack(layers, M: int, workspace: torch.Tensor | None = None, stream=None,
+                    path: int = OB_PATH_AUTO) -> None:
+    """Run a list of OneBit layers (M <= 16 tokens) in one persistent launch.
+
+    layers: sequence of (X, W_packed, a, b, Y, after_previous); X bf16 [M, K], W_packed int32
+    [N, K/32], a fp32 [N], b fp32 [K] or None, Y bf16/fp32 [M, N] (written), after_previous:
+    True if X is an output of an earlier layer of the list.  path: OB_PATH_AUTO,
+    OB_PATH_MMA_DECODE or OB_PATH_I8 (M <= 2).  workspace: at least ob_stack_workspace_size()
+    bytes; ob_linear_stack_workspace_size(layers, M) bytes enable the dataflow form.
+    """
+    arr, dev = _stack_array(layers, M)
     if workspace is None:
         workspace = torch.zeros(ob_stack_workspace_size(), dtype=torch.uint8, device=dev or "cuda")
     st = _lib.lib().ob_linear_stack_ex(arr, len(layers), M, _ptr(workspace), workspace.numel(), int(path),

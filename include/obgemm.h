@@ -252,8 +252,21 @@ typedef struct ob_layer {
 OB_API size_t ob_stack_workspace_size(void);
 
 /*
+ * Bytes of device workspace with which ob_linear_stack runs this list in its dataflow form:
+ * ob_stack_workspace_size() plus M x N x 4 bytes for every layer whose output a later layer
+ * of the same launch reads.  In that form (int8, M <= 2) a layer also writes its output as
+ * tagged 32-bit words, and a layer that reads it polls those words instead of waiting at a
+ * grid barrier.  The list qualifies when every layer writes its own buffer (no two outputs
+ * overlap) and every input is either outside all outputs of the list or exactly the bf16
+ * output of an earlier layer; otherwise (and for M > 2) this returns
+ * ob_stack_workspace_size(), and the list runs with grid barriers.  The library zeroes the
+ * tag area before every launch.
+ */
+OB_API size_t ob_linear_stack_workspace_size(const ob_layer* layers, int n_layers, int64_t M);
+
+/*
  * A list of OneBit layers at M <= 16 tokens (decode) in one persistent cooperative
- * launch per 384 layers, instead of one launch per layer: a decoder's layers read
+ * launch per 320 layers, instead of one launch per layer: a decoder's layers read
  * one another's outputs, and per-layer launches pay a launch and a drain for each.
  * The layers between two after_previous flags run back to back; a flagged layer
  * waits at a grid-wide barrier (bounded: a wait that runs out records
@@ -262,7 +275,9 @@ OB_API size_t ob_stack_workspace_size(void);
  *   layers     HOST array of n_layers descriptors (read during the call only).
  *   M          tokens, 0 <= M <= 16 (OB_ERR_SHAPE above).
  *   workspace  device, at least ob_stack_workspace_size() bytes, not shared with a
- *              concurrently running ob_linear_stack.
+ *              concurrently running ob_linear_stack; with
+ *              ob_linear_stack_workspace_size(layers, n_layers, M) bytes a qualifying list
+ *              runs in the dataflow form (no grid barriers).
  * Weights and scales must not be outputs of layers of the same list.  Validation of
  * every descriptor happens before anything is launched.  Asynchronous.
  * Kernel (OB_PATH_AUTO): M <= 2, the int8 form (one contiguous range of 16-row tiles

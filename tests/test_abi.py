@@ -164,6 +164,49 @@ def test_layernorm_and_stack_argument_checks_without_gpu(lib):
     assert st not in (NULL, SHAPE, ALIGN, WS, UNSUP)
 
 
+def test_stack_dataflow_workspace_analysis_without_gpu(lib):
+    # The dataflow form of ob_linear_stack (tagged outputs instead of grid barriers) needs every
+    # layer to write its own buffer and every input to be outside all outputs or exactly an
+    # earlier layer's bf16 output; otherwise the size is the barrier-only size.
+    from binary_weight_gemm_b200._lib import ObLayer
+    base = lib.ob_stack_workspace_size()
+
+    def size(descs, M):
+        arr = (ObLayer * len(descs))()
+        for i, d in enumerate(descs):
+            arr[i] = ObLayer(*d)
+        return lib.ob_linear_stack_workspace_size(arr, len(descs), M)
+
+    def align256(x):
+        return (x + 255) // 256 * 256
+
+    X0, W, A = 1 << 20, 2 << 20, 3 << 20
+    Y = [(8 + i) << 20 for i in range(4)]  # distinct 1 MB buffers
+    # chain X0 -> Y0 -> Y1 -> Y2 (K = N = 64): Y0 and Y1 are read by later layers
+    chain = [(X0, W, A, None, Y[0], 64, 64, 0, 0), (Y[0], W, A, None, Y[1], 64, 64, 0, 1),
+             (Y[1], W, A, None, Y[2], 64, 64, 0, 1)]
+    assert size(chain, 1) == base + align256(2 * 64 * 4)
+    assert size(chain, 2) == base + align256(2 * 2 * 64 * 4)
+    assert size(chain, 3) == base                       # the int8 form takes one or two tokens
+    # q, k, v read one input; o reads q: only q's output is tagged
+    block = [(X0, W, A, None, Y[0], 64, 128, 0, 0), (X0, W, A, None, Y[1], 64, 128, 0, 0),
+             (X0, W, A, None, Y[2], 64, 128, 0, 0), (Y[0], W, A, None, Y[3], 128, 64, 0, 1)]
+    assert size(block, 1) == base + align256(128 * 4)
+    # every tagged output starts on 256 bytes: 128 words each for two 96-wide outputs at M = 1
+    odd = [(X0, W, A, None, Y[0], 64, 96, 0, 0), (X0, W, A, None, Y[1], 64, 96, 0, 0),
+           (Y[0], W, A, None, Y[2], 96, 32, 0, 1), (Y[1], W, A, None, Y[3], 96, 32, 0, 1)]
+    assert size(odd, 1) == base + 2 * 512
+    # two layers writing one buffer, a later layer writing an earlier layer's input, an input
+    # that only overlaps an output, a producer with fp32 output: barriers only
+    assert size([chain[0], (Y[0], W, A, None, Y[0], 64, 64, 0, 1)], 1) == base
+    assert size([(X0, W, A, None, Y[0], 64, 64, 0, 0), (Y[0], W, A, None, X0, 64, 64, 0, 1)], 1) == base
+    assert size([chain[0], (Y[0] + 64, W, A, None, Y[1], 32, 64, 0, 1)], 1) == base
+    assert size([(X0, W, A, None, Y[0], 64, 64, 1, 0), (Y[0], W, A, None, Y[1], 64, 64, 0, 1)], 1) == base
+    # no consumer inside the list: nothing to tag
+    assert size([chain[0]], 1) == base
+    assert lib.ob_linear_stack_workspace_size(None, 3, 1) == base
+
+
 def test_factorize_argument_checks_without_gpu(lib):
     NULL, SHAPE, ALIGN, WS, UNSUP = 1, 2, 3, 6, 9
     p = ctypes.c_void_p(4096)
