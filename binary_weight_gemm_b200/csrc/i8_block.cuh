@@ -186,8 +186,11 @@ __device__ __forceinline__ void stage_pair(const StageRaw& raw, int m, const Sta
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     tpart += __shfl_xor_sync(0xffffffffu, tpart, o);
   }
+  // sigma = 2^sg with sg = 19 - e keeps max |q| < 2^20; sg in [-108, 126] keeps sigma and the
+  // fold factors 2^(1 + 7 l - sg) normal floats.  Only a pair whose largest |x'| is below
+  // 2^-107 (sub-normal range) keeps fewer than 20 bits.
   const int e = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127 : 0;
-  const int sg = max(-100, min(100, 19 - (e < -126 ? -126 : e)));
+  const int sg = max(-108, min(126, 19 - (e < -126 ? -126 : e)));
   const int q = lane >> 1, jh = (lane & 1) * 4;
   const int t = q >> 2, ee = q & 3, p = ee >> 1, half = ee & 1;
   const float sigma = pow2(sg);
