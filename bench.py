@@ -722,9 +722,9 @@ def run_stack(args, world, rank, local):
     specs = {m: spec(m) for m in ms_list}
     ws = torch.zeros(ops.ob_stack_workspace_size(), dtype=torch.uint8, device=dev)
 
-    # The dataflow form (int8, M <= 2): every layer of every block writes its own buffer, so
+    # The dataflow form (int8, one token): every layer of every block writes its own buffer, so
     # the list qualifies; consumers poll their producers' tagged outputs, no grid barriers.
-    df_ms = [m for m in ms_list if m <= 2]
+    df_ms = [m for m in ms_list if m == 1]
 
     def spec_df(m):
         x0, _ = acts[m]

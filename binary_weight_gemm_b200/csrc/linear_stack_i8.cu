@@ -25,6 +25,12 @@
 //  * The barrier is the bounded grid barrier of stack_common.cuh; the copy waits are
 //    bounded mbarrier waits.  Either running out records OB_ERR_DEVICE_TIMEOUT and ends
 //    the launch.
+//  * Dataflow launches (p.dataflow, one token, lists whose layers each write their own
+//    buffer): no grid barrier.  A layer whose output a later layer reads also stores it as
+//    32-bit words kTagMark | bf16 bits in a tag area the host zeroed before the launch; the
+//    consumer's staging polls those words (bounded, with back-off) until all of its pairs'
+//    words carry the mark, so it starts as soon as its own input is complete, one L2 round
+//    trip after the last producer's store instead of a barrier and a load.
 #include <algorithm>
 #include <cstring>
 
@@ -339,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_stack_i8_kernel(const __grid
                   break;
                 }
               }
-              __nanosleep(32);
+              __nanosleep(it < 4 ? 64 : 256);
             }
             if (!in_ok && lane == 0) s_abort = 1;
           } else {

@@ -101,7 +101,7 @@ cudaError_t launch_sign_stack(const StackLayerHost* layers, int n, int64_t M, un
                               int path, uint32_t* tags = nullptr, size_t tag_words = 0);
 int stack_max_layers_per_launch();
 // 32-bit words of tagged outputs a dataflow launch of the list needs (the largest over its
-// launches), or 0 when no launch of it qualifies: every layer writes its own buffer, and
+// launches), or 0 when no launch of it qualifies (one token only): every layer writes its own buffer, and
 // every input is either outside all outputs of its launch or exactly the bf16 output of an
 // earlier layer of it.
 size_t stack_tag_words(const StackLayerHost* layers, int n, int64_t M);

@@ -254,11 +254,11 @@ OB_API size_t ob_stack_workspace_size(void);
 /*
  * Bytes of device workspace with which ob_linear_stack runs this list in its dataflow form:
  * ob_stack_workspace_size() plus M x N x 4 bytes for every layer whose output a later layer
- * of the same launch reads.  In that form (int8, M <= 2) a layer also writes its output as
+ * of the same launch reads.  In that form (int8, M == 1) a layer also writes its output as
  * tagged 32-bit words, and a layer that reads it polls those words instead of waiting at a
  * grid barrier.  The list qualifies when every layer writes its own buffer (no two outputs
  * overlap) and every input is either outside all outputs of the list or exactly the bf16
- * output of an earlier layer; otherwise (and for M > 2) this returns
+ * output of an earlier layer; otherwise (and for M > 1) this returns
  * ob_stack_workspace_size(), and the list runs with grid barriers.  The library zeroes the
  * tag area before every launch.
  */

@@ -66,6 +66,8 @@ def _run(ops, spec, M, path=0, dataflow=False):
         n = ops.ob_linear_stack_workspace_size(spec, M)
         assert n > ops.ob_stack_workspace_size()
         ws = Guarded((n,), torch.uint8)
+    elif M == 2:  # two tokens keep the grid barriers whatever the workspace
+        assert ops.ob_linear_stack_workspace_size(spec, M) == ops.ob_stack_workspace_size()
     ops.ob_linear_stack(spec, M, path=path, workspace=None if ws is None else ws.t)
     torch.cuda.synchronize()
     assert ops.ob_last_device_error() == 0
@@ -74,7 +76,7 @@ def _run(ops, spec, M, path=0, dataflow=False):
 
 
 @pytest.mark.parametrize("M,path,df", [(1, 0, False), (2, 0, False), (4, 0, False), (9, 0, False), (16, 0, False),
-                                       (1, MMA, False), (2, MMA, False), (1, 0, True), (2, 0, True)])
+                                       (1, MMA, False), (2, MMA, False), (1, 0, True)])
 def test_stack_chain(ops, M, path, df):
     K = 512
     host = [_layer(200 + i, K, K) for i in range(8)]
@@ -90,7 +92,7 @@ def test_stack_chain(ops, M, path, df):
     _check(host, [(s[0], s[4]) for s in spec], f"chain M={M} path={path} dataflow={df}")
 
 
-@pytest.mark.parametrize("M,df", [(1, False), (2, False), (1, True), (2, True)])
+@pytest.mark.parametrize("M,df", [(1, False), (2, False), (1, True)])
 def test_stack_i8_tiles_chunks_and_tails(ops, M, df):
     # int8 form.  Group 1 (all read X0, K = 128): 60 layers of 32 rows (a CTA's tile range
     # crosses layers; the first writes fp32), one of 30000 rows (about 12.7 tiles per CTA:
@@ -119,7 +121,7 @@ def test_stack_i8_tiles_chunks_and_tails(ops, M, df):
     _check(host, [(sp[0], sp[4]) for sp in spec], f"i8 stack M={M} dataflow={df}")
 
 
-@pytest.mark.parametrize("M,df", [(1, False), (2, False), (5, False), (16, False), (1, True), (2, True)])
+@pytest.mark.parametrize("M,df", [(1, False), (2, False), (5, False), (16, False), (1, True)])
 def test_stack_groups_ragged(ops, M, df):
     # Group 1 (independent, all read X0): A 96->224, B 96->130 (fp32 out), C 96->64 without input
     # scale.  Group 2 (after a barrier): D reads A (224->200), E reads A too (224->128, vector path).
@@ -141,8 +143,7 @@ def test_stack_groups_ragged(ops, M, df):
     _check([host[n] for n, _, _ in shapes], [(src[n], out[n]) for n, _, _ in shapes], f"groups M={M} dataflow={df}")
 
 
-@pytest.mark.parametrize("M,path,df", [(1, 0, False), (2, 0, False), (16, 0, False), (1, MMA, False), (1, 0, True),
-                                       (2, 0, True)])
+@pytest.mark.parametrize("M,path,df", [(1, 0, False), (2, 0, False), (16, 0, False), (1, MMA, False), (1, 0, True)])
 def test_stack_dbf(ops, M, path, df):
     # DBF as two layers: T = ((X ⊙ b) S_B^T) ⊙ m, then Y = (T S_A^T) ⊙ a (no input scale).
     f = synth.dbf_factors(220, 1024, 512, 768)
@@ -185,7 +186,7 @@ def test_stack_longer_than_one_launch(ops, M, df):
                           what=f"long stack layer {i}")
 
 
-@pytest.mark.parametrize("M,df", [(1, False), (4, False), (1, True), (2, True)])
+@pytest.mark.parametrize("M,df", [(1, False), (4, False), (1, True)])
 def test_stack_in_cuda_graph(ops, M, df):
     # Replayed twice: the dataflow form's tag area is cleared inside the graph before each launch.
     K = 512
@@ -216,8 +217,8 @@ def test_stack_in_cuda_graph(ops, M, df):
     _check(host, [(sp[0], sp[4]) for sp in spec], "graph stack")
 
 
-@pytest.mark.parametrize("M,path,df", [(1, 0, False), (1, MMA, False), (2, 0, False), (16, 0, False), (1, 0, True),
-                                       (2, 0, True)], ids=["M1", "M1-mma", "M2", "M16", "M1-dataflow", "M2-dataflow"])
+@pytest.mark.parametrize("M,path,df", [(1, 0, False), (1, MMA, False), (2, 0, False), (16, 0, False), (1, 0, True)],
+                         ids=["M1", "M1-mma", "M2", "M16", "M1-dataflow"])
 def test_stack_7b_block(ops, M, path, df):
     # One 7B-shaped block: q, k, v, o (4096 -> 4096), gate, up (4096 -> 11008), down (11008 -> 4096).
     Wq, aq, bq, _ = oracle_svid(1, 4096, 4096)
