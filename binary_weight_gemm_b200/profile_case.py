@@ -4,7 +4,7 @@
     python -m binary_weight_gemm_b200.profile_case prefill --reps 6
     python -m binary_weight_gemm_b200.profile_case dbf --m 512 --reps 6
     python -m binary_weight_gemm_b200.profile_case dbf --m 1 --reps 20 --static [--path stack]
-    python -m binary_weight_gemm_b200.profile_case stack --m 1 --blocks 8 --reps 5
+    python -m binary_weight_gemm_b200.profile_case stack --m 1 --blocks 8 --reps 5 [--dataflow]
     python -m binary_weight_gemm_b200.profile_case stack --m 1 --chain 128 --reps 5 --path i8
 
 The workloads are the benchmark's: OneBit 4096 x 4096 decode at M tokens, OneBit
@@ -50,6 +50,8 @@ def main(argv=None) -> None:
     ap.add_argument("--path", choices=("auto", "mma", "i8", "stack"), default="auto",
                     help="stack / decode / dbf: kernel form (AUTO, the bf16 warp MMA, the int8 form; dbf also "
                          "'stack': both products in one persistent launch)")
+    ap.add_argument("--dataflow", action="store_true",
+                    help="stack: the workspace of ob_linear_stack_workspace_size (tagged outputs, no grid barriers)")
     ap.add_argument("--static", action="store_true",
                     help="decode / dbf: OR OB_FLAG_STATIC_WEIGHTS into the path (as the benchmark's decode calls do)")
     args = ap.parse_args(argv)
@@ -102,7 +104,9 @@ def main(argv=None) -> None:
             if name in ("down",) or args.chain:
                 x = Y
         desc = {"layers": len(spec), "blocks": 0 if args.chain else args.blocks}
-        ws = torch.zeros(ops.ob_stack_workspace_size(), dtype=torch.uint8, device=dev)
+        nws = ops.ob_linear_stack_workspace_size(spec, M) if args.dataflow else ops.ob_stack_workspace_size()
+        ws = torch.zeros(nws, dtype=torch.uint8, device=dev)
+        desc["dataflow"] = nws > ops.ob_stack_workspace_size()
         n_sets = 1
 
         def call(i):
