@@ -6,13 +6,14 @@
 // b folded into the sign operand as in linear_tc.cu.
 //
 // The same warp roles as linear_tc.cu, on a 2-CTA cluster that computes a 256 weight
-// rows x 256 tokens tile with M = 256 MMAs issued by rank 0:
+// rows x kTok tokens tile (kTok = 256, or 128 when the output has few tiles) with
+// M = 256 MMAs issued by rank 0:
 //  * each CTA expands its own 128 weight rows into its TMEM (rows 0..127 of the MMA's
-//    A in rank 0, 128..255 in rank 1) and loads its own 128 tokens of the activation
-//    tile (half of the MMA's N) by TMA, so per SM the activation traffic from L2 and
-//    the shared-memory reads of the MMA are half those of the one-CTA kernel;
+//    A in rank 0, 128..255 in rank 1) and loads its own kTok / 2 tokens of the
+//    activation tile (half of the MMA's N) by TMA, so per SM the activation traffic from
+//    L2 and the shared-memory reads of the MMA are half those of the one-CTA kernel;
 //  * a stage holds 128 k (two 64-k slabs of 128-byte-swizzled rows), 8 MMAs of
-//    256 x 256 x 16, so the per-stage hand-off is amortised over twice the math;
+//    256 x kTok x 16, so the per-stage hand-off is amortised over more math;
 //  * rank 0's `full` barrier receives both CTAs' TMA bytes and the arrivals of both
 //    CTAs' expansion warps; the MMA thread's commits arrive on the `empty` / `dfull`
 //    barriers of both CTAs; both epilogues release the accumulator on rank 0's
@@ -33,21 +34,31 @@ namespace ob {
 namespace {
 
 constexpr int kRowsCta = 128;   // weight rows per CTA (MMA M = 256 per pair)
-constexpr int kTok = 256;       // MMA N (tokens per pair tile)
-constexpr int kTokCta = 128;    // tokens loaded by each CTA
 constexpr int kBK = 128;        // k per stage
-constexpr int kStages = 4;
 constexpr int kThreads = 448;   // 14 warps
-constexpr uint32_t kSlabBytes = kTokCta * 64 * 2;         // 16 KB: 128 tokens x 64 k
-constexpr uint32_t kStageBytes = 2 * kSlabBytes;          // 32 KB per CTA
-constexpr uint32_t kOutTileBytes = kTok * kRowsCta * 2;   // 64 KB bf16 output tile
-constexpr int kTmemCols = 512;                            // D [0,256), A slots 256 + 64*s
-constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kRowsCta, kTok);
+constexpr int kTmemCols = 512;  // D [0, kTok), A slots kTok + 64*s
 constexpr int64_t kMaxK = 16384;
 // Warp roles: 0-7 expand signs (two per TMEM lane quadrant, each half of a stage's
 // 64 columns), 8-11 epilogue (one per quadrant), 12 TMA, 13 MMA (rank 0) + TMEM.
 constexpr int kAWarps = 8, kEpiWarps = 4, kEpiWarp0 = 8, kTmaWarp = 12, kMmaWarp = 13;
 
+// Tile shapes: kTok tokens per pair tile (MMA N), 256 or 128.  The narrow tile doubles
+// the number of tiles of an output with few of them (e.g. M = 512); its accumulator
+// takes 128 TMEM columns, which leaves room for six A stages instead of four.
+template <int kTok>
+struct Tc2Shape {
+  static constexpr int kTokCta = kTok / 2;                         // tokens loaded by each CTA
+  static constexpr int kStages = kTok == 256 ? 4 : 6;
+  static constexpr uint32_t kSlabBytes = kTokCta * 64 * 2;         // kTokCta tokens x 64 k
+  static constexpr uint32_t kStageBytes = 2 * kSlabBytes;          // per CTA
+  static constexpr uint32_t kOutTileBytes = kTok * kRowsCta * 2;   // bf16 output tile
+  static constexpr uint32_t kASlot0 = kTok;                        // TMEM column of A slot 0
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kRowsCta, kTok);
+  static_assert(kTok == 256 || kTok == 128, "pair tile of 256 or 128 tokens");
+  static_assert(kASlot0 + 64 * kStages <= kTmemCols, "accumulator and A stages fit TMEM");
+};
+
+template <int kStages>
 struct __align__(128) Tc2Shared {
   uint64_t full[kStages];  // rank 0: both CTAs' TMA bytes + 8 expansion warps + rank 0's TMA arrival
   uint64_t empty[kStages];  // both CTAs: the pair commit
@@ -75,15 +86,20 @@ __host__ __device__ __forceinline__ uint32_t unzip_bits2(uint32_t w) {
   return w;
 }
 
+template <int kTok>
 __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                      const __grid_constant__ CUtensorMap tmap_y,
                                                                      SignGemmArgs g, unsigned* err) {
+  using Sh = Tc2Shape<kTok>;
+  constexpr int kTokCta = Sh::kTokCta, kStages = Sh::kStages;
+  constexpr uint32_t kSlabBytes = Sh::kSlabBytes, kStageBytes = Sh::kStageBytes, kASlot0 = Sh::kASlot0;
+  using Shared = Tc2Shared<kStages>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // [ring: kStages x 32 KB][output tile 64 KB][Tc2Shared][iscale pairs]; the same
-  // offsets in both CTAs (the MMA reads B at one offset in each).
+  // [ring: kStages x kStageBytes][output tile][Shared][iscale pairs]; the same offsets in
+  // both CTAs (the MMA reads B at one offset in each).
   uint8_t* xs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* out_tile = xs + (size_t)kStages * kStageBytes;
-  Tc2Shared* sh = reinterpret_cast<Tc2Shared*>(out_tile + kOutTileBytes);
+  Shared* sh = reinterpret_cast<Shared*>(out_tile + Sh::kOutTileBytes);
   uint32_t* bpair = reinterpret_cast<uint32_t*>(sh + 1);  // [K/2] bf16x2 (iscale[2i], iscale[2i+1])
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -195,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
                 v[c] = cbase + e < valid ? (((u << (15 - (c & 15))) & 0x80008000u) ^ bb[e]) : 0u;
               }
             }
-            tmem_st_x32(lane_base + 256u + 64u * s + 32u * half, v);
+            tmem_st_x32(lane_base + kASlot0 + 64u * s + 32u * half, v);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -208,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
       }
     }
   } else if (warp < kEpiWarp0 + kEpiWarps) {
-    // ------------------------------------------------ epilogue: this CTA's 128 rows x 256 tokens
+    // ------------------------------------------------ epilogue: this CTA's 128 rows x kTok tokens
     const int q = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int c0 = 0, c1 = kTok / 32;
@@ -251,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
     }
     if (warp == kEpiWarp0 && lane == 0) bulk_wait_all();
   } else if (warp == kTmaWarp) {
-    // ------------------------------------------------ TMA producer: this CTA's 128 tokens
+    // ------------------------------------------------ TMA producer: this CTA's kTokCta tokens
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
       int64_t gstage = 0;
@@ -293,12 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
           if (!ok) break;
           tc_fence_after();
           const uint64_t so = (uint64_t)(s * (kStageBytes >> 4));
-          const uint32_t aa = tmem + 256u + 64u * s;
+          const uint32_t aa = tmem + kASlot0 + 64u * s;
           const int64_t rem = K - (int64_t)kb * kBK;
           const int steps = rem >= kBK ? 8 : (int)(rem / 16);  // K % 32 == 0: whole 16-k steps
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            if (j < steps) mma_bf16_ts_pair(tmem, aa + 8u * j, d[j] + so, kIdesc, (kb > 0 || j > 0) ? 1u : 0u);
+            if (j < steps) mma_bf16_ts_pair(tmem, aa + 8u * j, d[j] + so, Sh::kIdesc, (kb > 0 || j > 0) ? 1u : 0u);
           mma_commit_pair(&sh->empty[s]);
           if (++s == (uint32_t)kStages) {
             s = 0;
@@ -331,18 +347,18 @@ bool sign_gemm_tc2_supported(const SignGemmArgs& g) {
          (reinterpret_cast<uintptr_t>(g.Y) & 15) == 0;
 }
 
-cudaError_t launch_sign_gemm_tc2(const SignGemmArgs& g, const LaunchCtx& c) {
-  if (g.M == 0 || g.R == 0 || g.K == 0) return cudaSuccess;
-  if (!sign_gemm_tc2_supported(g)) return cudaErrorInvalidValue;
-  EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(tensor_map_encode_tiled_fn());
-  if (!encode) return cudaErrorNotSupported;
+namespace {
+
+template <int kTok>
+cudaError_t launch_tc2(const SignGemmArgs& g, const LaunchCtx& c, EncodeTiledFn encode) {
+  using Sh = Tc2Shape<kTok>;
   CUtensorMap tmap_x, tmap_y;
   std::memset(&tmap_x, 0, sizeof(tmap_x));
   std::memset(&tmap_y, 0, sizeof(tmap_y));
   {
     const cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.M};
     const cuuint64_t strides[1] = {(cuuint64_t)g.K * 2};
-    const cuuint32_t box[2] = {64u, (cuuint32_t)kTokCta};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)Sh::kTokCta};
     const cuuint32_t estr[2] = {1, 1};
     if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(g.X), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -361,8 +377,8 @@ cudaError_t launch_sign_gemm_tc2(const SignGemmArgs& g, const LaunchCtx& c) {
   }
   const int64_t tiles = ((g.M + kTok - 1) / kTok) * ((g.R + 2 * kRowsCta - 1) / (2 * kRowsCta));
   const int pairs = (int)std::min<int64_t>(tiles, c.num_sms / 2);
-  const size_t smem = 1024 + (size_t)kStages * kStageBytes + kOutTileBytes + sizeof(Tc2Shared) +
-                      sizeof(uint32_t) * ((((g.K + 1) / 2) + 3) & ~int64_t(3));
+  const size_t smem = 1024 + (size_t)Sh::kStages * Sh::kStageBytes + Sh::kOutTileBytes +
+                      sizeof(Tc2Shared<Sh::kStages>) + sizeof(uint32_t) * ((((g.K + 1) / 2) + 3) & ~int64_t(3));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -381,11 +397,29 @@ cudaError_t launch_sign_gemm_tc2(const SignGemmArgs& g, const LaunchCtx& c) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e = cudaFuncSetAttribute(sign_gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(sign_gemm_tc2_kernel<kTok>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = cudaLaunchKernelEx(&cfg, sign_gemm_tc2_kernel, tmap_x, tmap_y, g, c.err);
+  e = cudaLaunchKernelEx(&cfg, sign_gemm_tc2_kernel<kTok>, tmap_x, tmap_y, g, c.err);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sign_gemm_tc2_narrow(const SignGemmArgs& g, int num_sms) {
+  const int64_t wide = ((g.M + 255) / 256) * ((g.R + 2 * kRowsCta - 1) / (2 * kRowsCta));
+  return 2 * wide <= num_sms / 2;
+}
+
+cudaError_t launch_sign_gemm_tc2(const SignGemmArgs& g, const LaunchCtx& c) {
+  if (g.M == 0 || g.R == 0 || g.K == 0) return cudaSuccess;
+  if (!sign_gemm_tc2_supported(g)) return cudaErrorInvalidValue;
+  EncodeTiledFn encode = reinterpret_cast<EncodeTiledFn>(tensor_map_encode_tiled_fn());
+  if (!encode) return cudaErrorNotSupported;
+  // 128-token tiles when twice as many tiles as the 256-token tiling has still fit one
+  // wave of SM pairs (the wide tiling would leave more than half of the pairs idle).
+  return sign_gemm_tc2_narrow(g, c.num_sms) ? launch_tc2<128>(g, c, encode) : launch_tc2<256>(g, c, encode);
 }
 
 }  // namespace ob

@@ -53,6 +53,8 @@ void* tensor_map_encode_tiled_fn();
 // K <= 16384, M >= 512, R >= 256.
 bool sign_gemm_tc2_supported(const SignGemmArgs& g);
 cudaError_t launch_sign_gemm_tc2(const SignGemmArgs& g, const LaunchCtx& c);
+// Whether launch_sign_gemm_tc2 takes 128-token pair tiles for this shape.
+bool sign_gemm_tc2_narrow(const SignGemmArgs& g, int num_sms);
 
 // Largest K the tcgen05 GEMM takes (its input-scale pairs live in shared memory).
 int64_t sign_gemm_tc_max_k();

@@ -72,8 +72,10 @@ def test_dbf_workload_full(ops, M, path):
 
 # Middle dimensions for about 0.5, 1.5, 1.8 and 2.3 bits per weight at K = N = 4096
 # (bits ~ r (K + N) / (N K)): non-uniform r per layer, with tile tails in both sign GEMMs.
+# At M = 512 both products of r <= 3680 run on the CTA-pair kernel's 128-token tiles; at
+# r = 4704 both are split over K on the one-CTA kernel.
 @pytest.mark.parametrize("r", [1056, 3072, 3680, 4704])
-@pytest.mark.parametrize("M", [1, 16, 300])
+@pytest.mark.parametrize("M", [1, 16, 300, 512])
 def test_dbf_general_r(ops, r, M):
     f = synth.dbf_factors(r + M, 4096, r, 4096)
     xb, x = synth.activations(r, M, 4096)

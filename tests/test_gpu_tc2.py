@@ -3,8 +3,11 @@
 OB_PATH_TC (and AUTO above 16 tokens) with bf16 output, M >= 512 and N >= 256 runs
 the pair kernel (OB_PATH_TC1 forces the one-CTA kernel); these shapes exercise its
 ragged tiles: N not a multiple of 256
-(a pair whose second CTA has no valid rows), M not a multiple of 256, K with a
-partial 128-k stage.
+(a pair whose second CTA has no valid rows), M not a multiple of the token tile, K with a
+partial 128-k stage.  On 148 SMs the pair kernel takes 128-token tiles when twice the
+256-token tiles fit the 74 SM pairs: every shape below up to (2048, 384, 1056) takes the
+narrow tiles (777 tokens: the last tile's second CTA loads no valid token), the last two
+the 256-token tiles.
 """
 import numpy as np
 import pytest
@@ -31,7 +34,7 @@ def _cuda(x):
 
 
 @pytest.mark.parametrize("M,N,K", [(512, 256, 128), (600, 300, 160), (777, 520, 96), (1030, 1000, 4096),
-                                   (2048, 384, 1056)])
+                                   (2048, 384, 1056), (2304, 4000, 544), (4100, 2600, 1056)])
 def test_tc2_shapes(ops, M, N, K):
     seed = M + N + K
     W = synth.weights(seed, N, K)
