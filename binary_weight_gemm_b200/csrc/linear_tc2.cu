@@ -86,6 +86,30 @@ __host__ __device__ __forceinline__ uint32_t unzip_bits2(uint32_t w) {
   return w;
 }
 
+// The 32 TMEM columns of one half stage (64 k) of one weight row: column c holds the
+// bf16x2 pair of k = 2c, 2c+1, the two signs (from the unzipped words: u0 for columns
+// 0..15, u1 for 16..31) on the sign bits of bf16x2(iscale[k], iscale[k+1]) from bp.
+// kTail: a trailing partial stage; columns at or past `valid` (counted from the stage's
+// first column; this half starts at cbase0) are zero.
+template <bool kTail>
+__device__ __forceinline__ void expand_half(uint32_t u0, uint32_t u1, const uint4* bp, int cbase0, int valid,
+                                            uint32_t (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int cbase = cbase0 + 4 * q;
+    uint4 b4 = make_uint4(0, 0, 0, 0);
+    if (!kTail || cbase < valid) b4 = bp[q];
+    const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = 4 * q + e;  // column within this half
+      const uint32_t u = c < 16 ? u0 : u1;
+      const uint32_t x = ((u << (15 - (c & 15))) & 0x80008000u) ^ bb[e];
+      v[c] = (!kTail || cbase + e < valid) ? x : 0u;
+    }
+  }
+}
+
 template <int kTok>
 __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                      const __grid_constant__ CUtensorMap tmap_y,
@@ -152,6 +176,19 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
     const bool vec = (Wd & 3) == 0;
     int64_t gstage = 0;
     bool ok = true;
+    // A stage's TMEM store is waited for (and the stage released to the MMA on rank 0's
+    // `full` barrier) only after the next stage's columns are computed, so the store's
+    // latency overlaps that arithmetic.
+    int pending = -1;
+    auto flush_pending = [&]() {
+      if (pending >= 0) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(full0 + 8u * pending);
+        pending = -1;
+      }
+    };
     for (int64_t tile = pair; tile < tiles && ok; tile += npairs) {
       const int64_t n = (tile % n_blocks) * (2 * kRowsCta) + rank * kRowsCta + aq * 32 + lane;
       const bool row_ok = n < g.R;
@@ -180,49 +217,39 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
         for (int i = 0; i < 2; ++i) {
           const int kb = grp * 2 + i;
           if (kb >= nkb) break;
+          // Columns c = 0..63 of the stage hold k = 2c, 2c+1; a trailing partial stage
+          // (K % 128 != 0) leaves the columns past K at zero.
+          const int64_t left = K - (int64_t)kb * kBK;
+          const int valid = (int)(left < kBK ? left : kBK) / 2;
+          const uint4* bp = reinterpret_cast<const uint4*>(bpair + (int64_t)kb * (kBK / 2)) + 8 * ahalf;
+          // Selects keep cur in registers (no runtime index into it).
+          const uint32_t wa = i ? (ahalf ? cur[6] : cur[4]) : (ahalf ? cur[2] : cur[0]);
+          const uint32_t wb = i ? (ahalf ? cur[7] : cur[5]) : (ahalf ? cur[3] : cur[1]);
+          const uint32_t u0 = unzip_bits2(wa), u1 = unzip_bits2(wb);
+          uint32_t v[32];
+          if (left >= kBK)
+            expand_half<false>(u0, u1, bp, 32 * ahalf, valid, v);
+          else
+            expand_half<true>(u0, u1, bp, 32 * ahalf, valid, v);
+          // The previous stage's store has had this stage's arithmetic to land: only now
+          // wait for it and release that stage to the MMA.
+          flush_pending();
           const int s = (int)(gstage % kStages);
           if (gstage >= kStages) {
             ok = wait_warp(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag, lane);
             if (!ok) break;
             tc_fence_after();
           }
-          // Columns c = 0..63 of the stage hold k = 2c, 2c+1; a trailing partial stage
-          // (K % 128 != 0) leaves the columns past K at zero.
-          const int64_t left = K - (int64_t)kb * kBK;
-          const int valid = (int)(left < kBK ? left : kBK) / 2;
-          const uint4* bp = reinterpret_cast<const uint4*>(bpair + (int64_t)kb * (kBK / 2));
-          {
-            const int half = ahalf;
-            // Selects keep cur in registers (no runtime index into it).
-            const uint32_t wa = i ? (half ? cur[6] : cur[4]) : (half ? cur[2] : cur[0]);
-            const uint32_t wb = i ? (half ? cur[7] : cur[5]) : (half ? cur[3] : cur[1]);
-            const uint32_t u0 = unzip_bits2(wa), u1 = unzip_bits2(wb);
-            uint32_t v[32];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int cbase = 32 * half + 4 * q;
-              uint4 b4 = make_uint4(0, 0, 0, 0);
-              if (cbase < valid) b4 = bp[8 * half + q];
-              const uint32_t bb[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int c = 4 * q + e;  // column within this half
-                const uint32_t u = c < 16 ? u0 : u1;
-                v[c] = cbase + e < valid ? (((u << (15 - (c & 15))) & 0x80008000u) ^ bb[e]) : 0u;
-              }
-            }
-            tmem_st_x32(lane_base + kASlot0 + 64u * s + 32u * half, v);
-          }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_remote(full0 + 8u * s);
+          tmem_st_x32(lane_base + kASlot0 + 64u * s + 32u * ahalf, v);
+          pending = s;
           ++gstage;
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
       }
+      flush_pending();  // the tile's last stage, before the next tile's sign loads
     }
+    flush_pending();
   } else if (warp < kEpiWarp0 + kEpiWarps) {
     // ------------------------------------------------ epilogue: this CTA's 128 rows x kTok tokens
     const int q = warp & 3;
