@@ -73,7 +73,7 @@ struct __align__(128) Tc2Shared {
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, unsigned* err, volatile int* abort_flag,
                                           int lane) {
   int okw = 1;
-  if (lane == 0) okw = mbar_wait(bar, parity, err, abort_flag) ? 1 : 0;
+  if (lane == 0) okw = mbar_wait_sleep(bar, parity, err, abort_flag) ? 1 : 0;
   return __shfl_sync(0xffffffffu, okw, 0) != 0;
 }
 
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
         for (int kb = 0; kb < nkb; ++kb, ++gstage) {
           const int s = (int)(gstage % kStages);
           if (gstage >= kStages) {
-            ok = mbar_wait(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag);
+            ok = mbar_wait_sleep(&sh->empty[s], (uint32_t)((gstage / kStages) - 1) & 1u, err, abort_flag);
             if (!ok) break;
           }
           if (rank == 0) mbar_arrive_expect_tx(&sh->full[s], 2 * kStageBytes);  // both CTAs' bytes

@@ -96,6 +96,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   return mbar_wait_limit(bar, parity, err, abort_flag, OB_WAIT_LIMIT_NS);
 }
 
+// try_wait with a suspend-time hint: the thread may be suspended until the phase
+// completes or about hint_ns nanoseconds pass, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for a thread off the critical path (a producer running ahead of its
+// consumer, an epilogue waiting for a whole tile): each try lets the hardware suspend it
+// for up to 20 us, so it does not take issue slots from the warps that compute while it
+// waits.  Abort and timeout are checked after every try.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, unsigned* err,
+                                                volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > OB_WAIT_LIMIT_NS || it > (1u << 30)) {
+      record_error(err, OB_DEVERR_TIMEOUT);
+      if (abort_flag) *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
