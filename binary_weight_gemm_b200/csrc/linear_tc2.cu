@@ -265,19 +265,38 @@ __global__ void __launch_bounds__(kThreads, 1) sign_gemm_tc2_kernel(const __grid
       const int64_t n0 = (tile % n_blocks) * (2 * kRowsCta) + rank * kRowsCta;
       const int64_t nr = n0 + q * 32 + lane;
       const float sc = nr < g.R ? __ldg(g.oscale + nr) : 0.f;
-#pragma unroll 1
-      for (int c = c0; c < c1; ++c) {
-        uint32_t d[32];
-        tmem_ld_x32(lane_base + 32u * c, d);
-        tmem_wait_ld();
-        if (c == c1 - 1) {  // this warp's last read of the accumulator
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_remote(dempty0);
-        }
+      // The accumulator is read in chunks of 32 columns, two buffers deep: the load of chunk
+      // c + 1 is in flight while chunk c is converted and staged, and the accumulator is
+      // released to the next tile's MMAs as soon as the last chunk has landed in registers
+      // (the MMA waits for that release at every tile boundary).
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(dempty0);
+      };
+      auto stage_chunk = [&](const uint32_t (&d)[32], int c) {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
           col[(32 * c + i) * kRowsCta] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(d[i]) * sc));
+      };
+      static_assert((kTok / 32) % 2 == 0, "chunks are taken in pairs");
+      uint32_t da[32], db[32];
+      tmem_ld_x32(lane_base + 32u * c0, da);
+      tmem_wait_ld_regs(da);
+#pragma unroll 1
+      for (int c = c0; c < c1; c += 2) {
+        // da holds chunk c; chunk c + 1 (< c1: the count is even) goes to db.
+        tmem_ld_x32(lane_base + 32u * (c + 1), db);
+        stage_chunk(da, c);
+        tmem_wait_ld_regs(db);
+        if (c + 2 < c1) {
+          tmem_ld_x32(lane_base + 32u * (c + 2), da);
+          stage_chunk(db, c + 1);
+          tmem_wait_ld_regs(da);
+        } else {
+          release();  // this warp's last read of the accumulator has completed
+          stage_chunk(db, c + 1);
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
