@@ -114,19 +114,24 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 // consumer, an epilogue waiting for a whole tile): each try lets the hardware suspend it
 // for up to 20 us, so it does not take issue slots from the warps that compute while it
 // waits.  Abort and timeout are checked after every try.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, unsigned* err,
-                                                volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_sleep_limit(uint64_t* bar, uint32_t parity, unsigned* err,
+                                                      volatile int* abort_flag, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
     if (abort_flag && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > OB_WAIT_LIMIT_NS || it > (1u << 30)) {
+    if (globaltimer_ns() - t0 > limit_ns || it > (1u << 30)) {
       record_error(err, OB_DEVERR_TIMEOUT);
       if (abort_flag) *abort_flag = 1;
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, unsigned* err,
+                                                volatile int* abort_flag) {
+  return mbar_wait_sleep_limit(bar, parity, err, abort_flag, OB_WAIT_LIMIT_NS);
 }
 
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {

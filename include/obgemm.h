@@ -426,10 +426,12 @@ OB_API ob_status dbf_linear_noalloc(const void* X, int64_t M, int64_t K,
 
 /*
  * Self-test of the bounded-wait machinery (no counterpart on the pages): one
- * CTA waits on a barrier that nothing completes, gives up after `limit_ns`
- * nanoseconds, records OB_ERR_DEVICE_TIMEOUT in the device error word and
- * returns.  Synchronises `stream`; returns what ob_last_device_error reports
- * (OB_ERR_DEVICE_TIMEOUT when the machinery works).
+ * CTA waits on a barrier that nothing completes, first with the suspending
+ * wait, then with the polling one, each giving up after `limit_ns` nanoseconds
+ * (capped at 1 s); the second records OB_ERR_DEVICE_TIMEOUT in the device error
+ * word and the kernel returns.  Synchronises `stream`; returns what
+ * ob_last_device_error reports (OB_ERR_DEVICE_TIMEOUT when the machinery works,
+ * OB_ERR_NAN if the suspending wait did not give up as it must).
  */
 OB_API ob_status ob_selftest_timeout(uint64_t limit_ns, void* stream);
 
