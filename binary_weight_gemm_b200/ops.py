@@ -164,7 +164,8 @@ def _stack_array(layers, M: int):
 
 def ob_linear_stack_workspace_size(layers, M: int) -> int:
     """Workspace bytes with which ob_linear_stack runs this list in its dataflow form (tagged
-    outputs instead of grid barriers; int8 form, M <= 2), or ob_stack_workspace_size()."""
+    outputs instead of grid barriers; int8 form, one token, every layer writing its own
+    buffer), or ob_stack_workspace_size() where that form does not apply."""
     arr, _ = _stack_array(layers, M)
     return int(_lib.lib().ob_linear_stack_workspace_size(arr, len(layers), M))
 
